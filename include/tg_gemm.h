@@ -1,0 +1,152 @@
+/*
+ * tg_gemm.h -- C ABI of the tiled dense GEMM library for one NVIDIA B200.
+ *
+ * Operation (every entry point):
+ *
+ *     C[i][j] = epi( sum_{k<K} A[i][k] * B[k][j] ),   0 <= i < M, 0 <= j < N
+ *
+ * with A (M x K), B (K x N) and C (M x N) all ROW-MAJOR, i.e. element (r, c)
+ * of a matrix with leading dimension ld lives at base[r * ld + c].  This is
+ * the tiled matrix multiply of "TileLang ... 高效 GEMM 内核" (mhpq.cn),
+ * section 3.2 (C = A x B, A M x K, B K x N, fp32, caller-allocated C) and
+ * section 2.1 (tiling rationale); the row-major default is stated on the
+ * gtnt.cn TileLang tutorial, section 4.3; epi is the identity or the ReLU
+ * output post-processing of the blog.hotdry.top TileLang guide (landing
+ * checklist, item 2).  C is overwritten (no alpha/beta, no accumulation).
+ * Products are accumulated in fp32; the result is rounded once to C's type
+ * with round-to-nearest-even after epi is applied.
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ * - Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
+ *   current CUDA device.  The caller owns every buffer.  C must not overlap
+ *   A, B or the scales (not checked).
+ * - Leading dimensions are in elements (in bytes for the packed 4-bit
+ *   weight), and must be >= the row length.
+ * - stream is a cudaStream_t passed as void*; NULL means the legacy default
+ *   stream.  Calls are asynchronous: they validate, enqueue and return.
+ * - Sizes: M, N, K >= 0.  M == 0 or N == 0 -> TG_OK, nothing is launched.
+ *   K == 0 -> C = epi(0) = 0 is written.
+ * - Alignment (the hardware tensor-copy engine, TMA, needs 16-byte aligned
+ *   bases and row pitches): every base pointer 16-byte aligned and every
+ *   ld * sizeof(element) a multiple of 16 bytes, else TG_ERR_ALIGNMENT.
+ * - Errors are returned, never printed or thrown.  Validation happens
+ *   before any CUDA call; on any error nothing is launched and C is untouched.
+ * - The library allocates no per-call memory.  It keeps, per device and for
+ *   the life of the process, a small status word (see
+ *   tg_last_device_status) and a cache of tensor-copy descriptors.
+ * - Thread safety: calls from several host threads are allowed.
+ */
+#ifndef TG_GEMM_H
+#define TG_GEMM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,  /* negative size, NULL pointer, ld < row length, bad flag */
+    TG_ERR_ALIGNMENT = 2,    /* base not 16-byte aligned or row pitch not a multiple of 16 bytes */
+    TG_ERR_UNSUPPORTED = 3,  /* group size other than 128, K not a multiple of it, size limit */
+    TG_ERR_CUDA = 4,         /* a CUDA runtime / driver call or the launch failed */
+    TG_ERR_TIMEOUT = 5,      /* a kernel's bounded wait expired (reported by tg_last_device_status) */
+    TG_ERR_NO_DEVICE = 6     /* no sm_100 device is current */
+} tg_status;
+
+/* Epilogue flags (the `epilogue` argument). */
+enum { TG_EPI_NONE = 0, TG_EPI_RELU = 1 };
+
+/* fp32 modes (the `mode` argument of tg_gemm_f32). */
+enum {
+    TG_F32_FFMA = 0,  /* exact fp32 products, fp32 FMA accumulation on CUDA cores */
+    TG_F32_TF32 = 1   /* operands rounded to TF32 (10-bit mantissa) by the tensor
+                         cores, fp32 accumulation in tensor memory */
+};
+
+/*
+ * tg_gemm_f32 -- fp32 GEMM (mhpq.cn article, section 3.2: float32 A, B, C,
+ * 128 x 128 x 32 tiles, 256 threads; section 3.3: float4 vector loads).
+ *   A: M x K floats, row pitch lda (>= K, lda % 4 == 0)
+ *   B: K x N floats, row pitch ldb (>= N, ldb % 4 == 0)
+ *   C: M x N floats, row pitch ldc (>= N, ldc % 4 == 0); written
+ *   epilogue: TG_EPI_NONE or TG_EPI_RELU; mode: TG_F32_FFMA or TG_F32_TF32
+ */
+tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K,
+                      const float *A, int64_t lda,
+                      const float *B, int64_t ldb,
+                      float *C, int64_t ldc,
+                      int epilogue, int mode, void *stream);
+
+/*
+ * tg_gemm_f16 -- fp16 operands and output, fp32 accumulation (explicit cast
+ * to float16, gtnt.cn tutorial section 4.3; FP16 GEMM on the blog.hotdry.top
+ * guide).  A, B, C hold IEEE binary16 values (e.g. __half or torch.float16);
+ * every ld must be a multiple of 8 elements.  Other arguments as tg_gemm_f32.
+ */
+tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K,
+                      const void *A, int64_t lda,
+                      const void *B, int64_t ldb,
+                      void *C, int64_t ldc,
+                      int epilogue, void *stream);
+
+/* tg_gemm_bf16 -- as tg_gemm_f16 with bfloat16 operands and output. */
+tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
+                       const void *A, int64_t lda,
+                       const void *B, int64_t ldb,
+                       void *C, int64_t ldc,
+                       int epilogue, void *stream);
+
+/*
+ * tg_gemm_w4a16 -- dequantize GEMM (the "Dequant GEMM" workload of the
+ * blog.hotdry.top TileLang guide; the pages give no format, this library
+ * defines it):  C = epi(A . W) with
+ *
+ *     W[k][n] = fp16( q[k][n] * s[k / group_size][n] )
+ *
+ *   A:      M x K fp16 activations, row pitch lda (elements, % 8 == 0)
+ *   Bq:     K rows of packed signed 4-bit weights q in [-8, 7], two's
+ *           complement, two per byte: column 2j in bits 0-3 and column 2j+1
+ *           in bits 4-7 of byte j of the row.  Row pitch ldbq in BYTES
+ *           (>= ceil(N/2), % 16 == 0).
+ *   scales: ceil(K / group_size) x N fp16 scales, row pitch lds (elements,
+ *           % 8 == 0).
+ *   group_size: must be 128, and K must be a multiple of it, else
+ *           TG_ERR_UNSUPPORTED.
+ *   C:      M x N fp16 output, row pitch ldc (elements, % 8 == 0).
+ * The dequantised weight is formed as an fp32 product rounded once to fp16
+ * (so it equals the exact product rounded to fp16), then used as an fp16
+ * tensor-core operand with fp32 accumulation.
+ */
+tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
+                        const void *A, int64_t lda,
+                        const uint8_t *Bq, int64_t ldbq,
+                        const void *scales, int64_t lds, int group_size,
+                        void *C, int64_t ldc,
+                        int epilogue, void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *tg_status_string(tg_status s);
+
+/*
+ * tg_last_device_status -- synchronises `stream`, then reads and clears the
+ * current device's status word.  Kernels never spin forever: every wait on
+ * a pipeline barrier has an iteration limit, and a kernel that hits it
+ * records TG_ERR_TIMEOUT there and returns early (C is then incomplete).
+ * Returns TG_OK, TG_ERR_TIMEOUT, or TG_ERR_CUDA if synchronising failed.
+ */
+tg_status tg_last_device_status(void *stream);
+
+/*
+ * tg_num_sms -- number of SMs of the current device (what the persistent
+ * kernels size their grids by), or -1 on error.
+ */
+int tg_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TG_GEMM_H */

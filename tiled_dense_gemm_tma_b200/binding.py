@@ -1,0 +1,167 @@
+"""ctypes binding of the C ABI declared in include/tg_gemm.h.
+
+Argument marshalling only: every step of the GEMM runs in the CUDA kernels
+of ``libtg_gemm.so``.  Torch is used for device memory and streams.  If the
+library is missing, the first call raises; there is no fallback.
+"""
+import ctypes
+import os
+import threading
+
+LIB_NAME = "libtg_gemm.so"
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+EPI_NONE, EPI_RELU = 0, 1
+F32_FFMA, F32_TF32 = 0, 1
+
+STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
+          3: "TG_ERR_UNSUPPORTED", 4: "TG_ERR_CUDA", 5: "TG_ERR_TIMEOUT",
+          6: "TG_ERR_NO_DEVICE"}
+
+# Every symbol include/tg_gemm.h declares.
+EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
+           "tg_status_string", "tg_last_device_status", "tg_num_sms")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class TgError(RuntimeError):
+    """A non-OK tg_status returned by the library."""
+
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+def lib_path():
+    return os.path.join(_HERE, LIB_NAME)
+
+
+def load_library():
+    """Load libtg_gemm.so (built in-tree) and declare its signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = lib_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{LIB_NAME} is not built (expected at {path}); "
+                              "run tiled_dense_gemm_tma_b200/build.py")
+        lib = ctypes.CDLL(path)
+        i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        lib.tg_gemm_f32.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, ci, vp]
+        for name in ("tg_gemm_f16", "tg_gemm_bf16"):
+            getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, vp]
+        lib.tg_gemm_w4a16.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
+                                      vp, i64, ci, vp]
+        for name in ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
+                     "tg_last_device_status"):
+            getattr(lib, name).restype = ci
+        lib.tg_status_string.argtypes = [ci]
+        lib.tg_status_string.restype = ctypes.c_char_p
+        lib.tg_last_device_status.argtypes = [vp]
+        lib.tg_num_sms.argtypes = []
+        lib.tg_num_sms.restype = ci
+        _lib = lib
+        return lib
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ld(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D")
+    if t.stride(1) != 1 and t.shape[1] > 1:
+        raise ValueError(f"{name} must be row-major (unit column stride)")
+    return max(t.stride(0), t.shape[1]) if t.shape[0] <= 1 else t.stride(0)
+
+
+def _check(code, what):
+    if code != 0:
+        raise TgError(code, what)
+
+
+def _mk(A, B, C, dtype, out_dtype):
+    import torch
+    M, K = A.shape
+    K2, N = B.shape
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: {K} vs {K2}")
+    for t, n in ((A, "A"), (B, "B")):
+        if t.dtype != dtype:
+            raise TypeError(f"{n} must be {dtype}")
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+    if C is None:
+        C = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    elif C.shape != (M, N) or C.dtype != out_dtype:
+        raise ValueError("C has the wrong shape or dtype")
+    return M, N, K, C
+
+
+def gemm_f32(A, B, C=None, relu=False, mode=F32_FFMA, stream=None):
+    """C = epi(A @ B) for float32 CUDA tensors; mode F32_FFMA or F32_TF32."""
+    import torch
+    lib = load_library()
+    M, N, K, C = _mk(A, B, C, torch.float32, torch.float32)
+    _check(lib.tg_gemm_f32(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
+                           C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                           mode, _stream_handle(stream)), "tg_gemm_f32")
+    return C
+
+
+def gemm_f16(A, B, C=None, relu=False, stream=None):
+    """C = epi(A @ B) for float16 CUDA tensors, fp32 accumulation."""
+    import torch
+    lib = load_library()
+    M, N, K, C = _mk(A, B, C, torch.float16, torch.float16)
+    _check(lib.tg_gemm_f16(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
+                           C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                           _stream_handle(stream)), "tg_gemm_f16")
+    return C
+
+
+def gemm_bf16(A, B, C=None, relu=False, stream=None):
+    """C = epi(A @ B) for bfloat16 CUDA tensors, fp32 accumulation."""
+    import torch
+    lib = load_library()
+    M, N, K, C = _mk(A, B, C, torch.bfloat16, torch.bfloat16)
+    _check(lib.tg_gemm_bf16(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
+                            C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                            _stream_handle(stream)), "tg_gemm_bf16")
+    return C
+
+
+def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None):
+    """C = epi(A @ W), W[k, n] = q[k, n] * scales[k // group_size, n].
+
+    A: M x K float16; Bq: K x ldbq uint8 (packed, low nibble = even column);
+    scales: (K // group_size) x N float16; N: number of output columns.
+    """
+    import torch
+    lib = load_library()
+    if A.dtype != torch.float16 or scales.dtype != torch.float16 or Bq.dtype != torch.uint8:
+        raise TypeError("A and scales must be float16, Bq uint8")
+    M, K = A.shape
+    if Bq.shape[0] != K:
+        raise ValueError("Bq must have K rows")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.tg_gemm_w4a16(M, N, K, A.data_ptr(), _ld(A, "A"), Bq.data_ptr(), _ld(Bq, "Bq"),
+                             scales.data_ptr(), _ld(scales, "scales"), group_size,
+                             C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                             _stream_handle(stream)), "tg_gemm_w4a16")
+    return C
+
+
+def last_device_status(stream=None):
+    """Synchronise the stream and return (and clear) the device status word."""
+    return load_library().tg_last_device_status(_stream_handle(stream))

@@ -1,0 +1,116 @@
+"""Seeded synthetic inputs for the GEMM paths.
+
+This module draws and stores input matrices; it holds none of the GEMM's
+arithmetic and imports neither the CUDA binding nor the oracle, so both
+sides of a parity test can take their inputs from here.
+
+Recipe (the pages fix no input data; the distributions are those of the
+library's benchmark workloads):
+
+* ``numpy.random.default_rng(seed)`` (PCG64) is the only source.  Draws are
+  made in the order A, then B (then q, then scales for the 4-bit path), each
+  matrix row-major in one call.
+* Real values are drawn in float64 and rounded once to the storage type:
+  float32 and float16 by numpy's round-to-nearest-even casts; bfloat16 by
+  rounding to float32 first and then to bfloat16 with round-to-nearest-even
+  on the bit pattern (so bf16 values are double-rounded through fp32; any
+  deterministic rounding serves, since both sides read the stored values).
+* fp16 / bf16 matrices are returned as uint16 bit-pattern arrays.
+* The 4-bit weight q (integers in [-8, 7]) is packed two per byte, column
+  2j in the low nibble and 2j+1 in the high nibble of byte j of its row.
+"""
+import math
+
+import numpy as np
+
+
+def _to_bf16_bits(x64):
+    f32 = np.asarray(x64, np.float64).astype(np.float32)
+    u = f32.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(f32)
+    if nan.any():
+        r[nan] = 0x7FC0
+    return r
+
+
+def _to_f16_bits(x64):
+    return np.asarray(x64, np.float64).astype(np.float16).view(np.uint16)
+
+
+def store(x64, dtype):
+    """Round float64 draws to a storage type: 'f32', 'f16' or 'bf16'."""
+    if dtype == "f32":
+        return np.asarray(x64, np.float64).astype(np.float32)
+    if dtype == "f16":
+        return _to_f16_bits(x64)
+    if dtype == "bf16":
+        return _to_bf16_bits(x64)
+    raise ValueError(dtype)
+
+
+def pack_int4(q):
+    """Pack an int array (K x N, values in [-8, 7]) into K x ceil(N/2) bytes."""
+    q = np.asarray(q)
+    if q.min(initial=0) < -8 or q.max(initial=0) > 7:
+        raise ValueError("q out of [-8, 7]")
+    K, N = q.shape
+    nib = (q.astype(np.int64) & 0xF).astype(np.uint8)
+    if N % 2:
+        nib = np.concatenate([nib, np.zeros((K, 1), np.uint8)], axis=1)
+    return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+
+
+def uniform_pm1(M, N, K, seed, dtype="f32"):
+    """A (M x K), B (K x N) with i.i.d. uniform[-1, 1] entries."""
+    rng = np.random.default_rng(seed)
+    A = rng.uniform(-1.0, 1.0, size=(M, K))
+    B = rng.uniform(-1.0, 1.0, size=(K, N))
+    return store(A, dtype), store(B, dtype)
+
+
+def normal(M, N, K, seed, dtype="f32", scale_by_sqrt_k=False):
+    """A, B with i.i.d. N(0, 1) entries, optionally divided by sqrt(K)."""
+    rng = np.random.default_rng(seed)
+    s = 1.0 / math.sqrt(K) if (scale_by_sqrt_k and K > 0) else 1.0
+    A = rng.standard_normal(size=(M, K)) * s
+    B = rng.standard_normal(size=(K, N)) * s
+    return store(A, dtype), store(B, dtype)
+
+
+def integers(M, N, K, seed, lo=-3, hi=3, dtype="f32"):
+    """A, B with i.i.d. integer entries uniform in {lo..hi}."""
+    rng = np.random.default_rng(seed)
+    A = rng.integers(lo, hi + 1, size=(M, K)).astype(np.float64)
+    B = rng.integers(lo, hi + 1, size=(K, N)).astype(np.float64)
+    return store(A, dtype), store(B, dtype)
+
+
+def w4a16(M, N, K, seed, group=128, s_lo=0.005, s_hi=0.02, a_int=None):
+    """Inputs of the 4-bit-weight GEMM.
+
+    Returns (A fp16 bits M x K, Bq packed uint8 K x ceil(N/2), scales fp16
+    bits ceil(K/group) x N, q int8 K x N).  A is N(0, 1), or integers in
+    [-a_int, a_int] when a_int is given; q is uniform in {-8..7}; scales are
+    uniform[s_lo, s_hi] rounded to fp16.
+    """
+    rng = np.random.default_rng(seed)
+    if a_int is None:
+        A = rng.standard_normal(size=(M, K))
+    else:
+        A = rng.integers(-a_int, a_int + 1, size=(M, K)).astype(np.float64)
+    q = rng.integers(-8, 8, size=(K, N)).astype(np.int8)
+    G = (K + group - 1) // group
+    s = rng.uniform(s_lo, s_hi, size=(G, N))
+    return store(A, "f16"), pack_int4(q), store(s, "f16"), q
+
+
+def with_ld(X, ld):
+    """Copy a 2-D array into a wider row pitch ld (extra columns zero)."""
+    R, C = X.shape
+    if ld < C:
+        raise ValueError("ld < columns")
+    out = np.zeros((R, ld), X.dtype)
+    out[:, :C] = X
+    return out[:, :C]
