@@ -42,6 +42,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TG_API __attribute__((visibility("default")))
+#else
+#define TG_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -74,7 +80,7 @@ enum {
  *   C: M x N floats, row pitch ldc (>= N, ldc % 4 == 0); written
  *   epilogue: TG_EPI_NONE or TG_EPI_RELU; mode: TG_F32_FFMA or TG_F32_TF32
  */
-tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K,
+TG_API tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K,
                       const float *A, int64_t lda,
                       const float *B, int64_t ldb,
                       float *C, int64_t ldc,
@@ -86,14 +92,14 @@ tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K,
  * guide).  A, B, C hold IEEE binary16 values (e.g. __half or torch.float16);
  * every ld must be a multiple of 8 elements.  Other arguments as tg_gemm_f32.
  */
-tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K,
+TG_API tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K,
                       const void *A, int64_t lda,
                       const void *B, int64_t ldb,
                       void *C, int64_t ldc,
                       int epilogue, void *stream);
 
 /* tg_gemm_bf16 -- as tg_gemm_f16 with bfloat16 operands and output. */
-tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
+TG_API tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
                        const void *A, int64_t lda,
                        const void *B, int64_t ldb,
                        void *C, int64_t ldc,
@@ -120,7 +126,7 @@ tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
  * (so it equals the exact product rounded to fp16), then used as an fp16
  * tensor-core operand with fp32 accumulation.
  */
-tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
+TG_API tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
                         const void *A, int64_t lda,
                         const uint8_t *Bq, int64_t ldbq,
                         const void *scales, int64_t lds, int group_size,
@@ -128,7 +134,7 @@ tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
                         int epilogue, void *stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
-const char *tg_status_string(tg_status s);
+TG_API const char *tg_status_string(tg_status s);
 
 /*
  * tg_last_device_status -- synchronises `stream`, then reads and clears the
@@ -137,13 +143,13 @@ const char *tg_status_string(tg_status s);
  * records TG_ERR_TIMEOUT there and returns early (C is then incomplete).
  * Returns TG_OK, TG_ERR_TIMEOUT, or TG_ERR_CUDA if synchronising failed.
  */
-tg_status tg_last_device_status(void *stream);
+TG_API tg_status tg_last_device_status(void *stream);
 
 /*
  * tg_num_sms -- number of SMs of the current device (what the persistent
  * kernels size their grids by), or -1 on error.
  */
-int tg_num_sms(void);
+TG_API int tg_num_sms(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/tg_gemm.h declares, and rejects bad arguments before
+touching CUDA (nothing is launched, so these run on a machine without GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tiled_dense_gemm_tma_b200 import binding, build as tg_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, ALIGN, UNSUP = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tg_build.build()
+    return binding.load_library()
+
+
+def test_header_symbols_exported(lib):
+    with open(os.path.join(ROOT, "include", "tg_gemm.h")) as f:
+        text = f.read()
+    declared = set(re.findall(r"\b(tg_\w+)\s*\(", text))
+    assert declared == set(binding.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert lib.tg_status_string(code).decode() == name
+    assert lib.tg_status_string(99).decode() == "TG_ERR_UNKNOWN"
+
+
+P = 0x10000          # a fake, 16-byte aligned "device" address (never dereferenced)
+
+
+def _bf16(lib, M, N, K, A=P, lda=None, B=P, ldb=None, C=P, ldc=None, epi=0):
+    lda = K if lda is None else lda
+    ldb = N if ldb is None else ldb
+    ldc = N if ldc is None else ldc
+    return lib.tg_gemm_bf16(M, N, K, A, lda, B, ldb, C, ldc, epi, None)
+
+
+def test_argument_validation_bf16(lib):
+    assert _bf16(lib, -1, 8, 8) == INVALID
+    assert _bf16(lib, 8, -1, 8) == INVALID
+    assert _bf16(lib, 8, 8, -1) == INVALID
+    assert _bf16(lib, 8, 8, 8, epi=2) == INVALID
+    assert _bf16(lib, 0, 8, 8) == OK               # empty output: nothing to do
+    assert _bf16(lib, 8, 0, 8) == OK
+    assert _bf16(lib, 8, 8, 8, A=None) == INVALID
+    assert _bf16(lib, 8, 8, 8, C=None) == INVALID
+    assert _bf16(lib, 8, 8, 8, lda=7) == INVALID
+    assert _bf16(lib, 8, 8, 8, ldc=4) == INVALID
+    assert _bf16(lib, 8, 8, 8, A=P + 8) == ALIGN
+    assert _bf16(lib, 8, 8, 8, C=P + 2) == ALIGN
+    assert _bf16(lib, 8, 12, 8, ldb=12, ldc=16) == ALIGN   # 24-byte row pitch
+    assert _bf16(lib, 8, 8, 8, lda=12) == ALIGN
+    assert _bf16(lib, 1 << 31, 8, 8) == UNSUP
+
+
+def test_argument_validation_f32_and_f16(lib):
+    f = lib.tg_gemm_f32
+    assert f(8, 8, 8, P, 8, P, 8, P, 8, 0, 2, None) == INVALID      # bad mode
+    assert f(8, 8, 8, P, 6, P, 8, P, 8, 0, 0, None) == INVALID      # lda < K
+    assert f(8, 8, 8, P, 10, P, 8, P, 8, 0, 0, None) == ALIGN       # 40-byte pitch
+    assert f(8, 0, 8, P, 8, P, 8, P, 8, 0, 1, None) == OK
+    g = lib.tg_gemm_f16
+    assert g(8, 8, 8, P, 8, P, 8, P + 4, 8, 0, None) == ALIGN
+    assert g(8, 8, 8, P, 8, None, 8, P, 8, 0, None) == INVALID
+
+
+def test_argument_validation_w4a16(lib):
+    w = lib.tg_gemm_w4a16
+    # M, N, K, A, lda, Bq, ldbq, scales, lds, group, C, ldc, epi, stream
+    assert w(4, 32, 256, P, 256, P, 16, P, 32, 64, P, 32, 0, None) == UNSUP     # group 64
+    assert w(4, 32, 200, P, 200, P, 16, P, 32, 128, P, 32, 0, None) == UNSUP    # K % 128
+    assert w(4, 32, 256, P, 256, P, 8, P, 32, 128, P, 32, 0, None) == INVALID   # ldbq < N/2
+    assert w(4, 32, 256, P, 256, P, 24, P, 32, 128, P, 32, 0, None) == ALIGN    # ldbq % 16
+    assert w(4, 32, 256, P, 256, P, 16, P + 2, 32, 128, P, 32, 0, None) == ALIGN
+    assert w(4, 32, 256, P, 256, P, 16, None, 32, 128, P, 32, 0, None) == INVALID
+    assert w(0, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 0, None) == OK
+    assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 3, None) == INVALID
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_HERE", str(tmp_path))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(ImportError):
+        binding.load_library()

@@ -1,0 +1,166 @@
+// abi.cu -- the C ABI of include/tg_gemm.h: argument validation and dispatch.
+//
+// Every check here runs before any CUDA call, so a rejected call has no side
+// effect.  The operation and its conventions are documented in the header.
+#include "../../include/tg_gemm.h"
+#include "launch.h"
+#include "host.cuh"
+#include "ptx.cuh"
+
+#include <cuda_runtime.h>
+
+namespace tg {
+
+// Per-device status word written by kernels whose bounded wait expired.
+__device__ int g_device_status = 0;
+
+int* device_status_ptr() {
+    static int* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int*>(p);
+    }
+    return ptrs[dev];
+}
+
+}  // namespace tg
+
+namespace {
+
+constexpr int64_t kMaxDim = (1ll << 31) - 1;      // kernel indices and TMA coords are int32
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared checks for a plain GEMM with element size `eb` (bytes).
+tg_status check_gemm(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                     const void* B, int64_t ldb, const void* C, int64_t ldc,
+                     int epilogue, int eb) {
+    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
+    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return TG_OK;
+    if (!C || ldc < N) return TG_ERR_INVALID_ARG;
+    if (K > 0 && (!A || !B || lda < K || ldb < N)) return TG_ERR_INVALID_ARG;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!aligned16(C) || (ldc * eb) % 16 != 0) return TG_ERR_ALIGNMENT;
+    if (K > 0 && (!aligned16(A) || !aligned16(B) || (lda * eb) % 16 != 0 || (ldb * eb) % 16 != 0))
+        return TG_ERR_ALIGNMENT;
+    // TMA strides must stay below 2^40 bytes.
+    if (ldc * eb >= (1ll << 40) || lda * eb >= (1ll << 40) || ldb * eb >= (1ll << 40))
+        return TG_ERR_UNSUPPORTED;
+    return TG_OK;
+}
+
+// C = epi(0) = 0 when K == 0.
+tg_status zero_fill(void* C, int64_t ldc, int64_t M, int64_t N, int eb, void* stream) {
+    int dev;
+    if (!tg::current_device(&dev)) return TG_ERR_NO_DEVICE;
+    cudaError_t e = cudaMemset2DAsync(C, static_cast<size_t>(ldc * eb), 0,
+                                      static_cast<size_t>(N * eb), static_cast<size_t>(M),
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+}
+
+tg::GemmArgs make_args(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                       const void* B, int64_t ldb, void* C, int64_t ldc, int epilogue,
+                       void* stream) {
+    tg::GemmArgs a;
+    a.M = M; a.N = N; a.K = K;
+    a.A = A; a.lda = lda; a.B = B; a.ldb = ldb; a.C = C; a.ldc = ldc;
+    a.scales = nullptr; a.lds = 0; a.group = 0;
+    a.relu = epilogue == TG_EPI_RELU;
+    a.stream = stream;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K, const float* A, int64_t lda,
+                      const float* B, int64_t ldb, float* C, int64_t ldc, int epilogue,
+                      int mode, void* stream) {
+    if (mode != TG_F32_FFMA && mode != TG_F32_TF32) return TG_ERR_INVALID_ARG;
+    tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 4);
+    if (s != TG_OK || M == 0 || N == 0) return s;
+    if (K == 0) return zero_fill(C, ldc, M, N, 4, stream);
+    tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
+    return static_cast<tg_status>(mode == TG_F32_TF32 ? tg::launch_tc_tf32(a)
+                                                      : tg::launch_ffma_f32(a));
+}
+
+tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                      const void* B, int64_t ldb, void* C, int64_t ldc, int epilogue,
+                      void* stream) {
+    tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2);
+    if (s != TG_OK || M == 0 || N == 0) return s;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    return static_cast<tg_status>(
+        tg::launch_tc_f16(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream)));
+}
+
+tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                       const void* B, int64_t ldb, void* C, int64_t ldc, int epilogue,
+                       void* stream) {
+    tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2);
+    if (s != TG_OK || M == 0 || N == 0) return s;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    return static_cast<tg_status>(
+        tg::launch_tc_bf16(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream)));
+}
+
+tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                        const uint8_t* Bq, int64_t ldbq, const void* scales, int64_t lds,
+                        int group_size, void* C, int64_t ldc, int epilogue, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
+    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if (group_size != 128 || K % 128 != 0) return TG_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return TG_OK;
+    if (!C || ldc < N) return TG_ERR_INVALID_ARG;
+    if (K > 0 && (!A || !Bq || !scales || lda < K || ldbq < (N + 1) / 2 || lds < N))
+        return TG_ERR_INVALID_ARG;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!aligned16(C) || (ldc * 2) % 16 != 0) return TG_ERR_ALIGNMENT;
+    if (K > 0 && (!aligned16(A) || !aligned16(Bq) || !aligned16(scales) || (lda * 2) % 16 != 0 ||
+                  ldbq % 16 != 0 || (lds * 2) % 16 != 0))
+        return TG_ERR_ALIGNMENT;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    tg::GemmArgs a = make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream);
+    a.scales = scales;
+    a.lds = lds;
+    a.group = group_size;
+    return static_cast<tg_status>(tg::launch_w4a16(a));
+}
+
+const char* tg_status_string(tg_status s) {
+    switch (s) {
+        case TG_OK: return "TG_OK";
+        case TG_ERR_INVALID_ARG: return "TG_ERR_INVALID_ARG";
+        case TG_ERR_ALIGNMENT: return "TG_ERR_ALIGNMENT";
+        case TG_ERR_UNSUPPORTED: return "TG_ERR_UNSUPPORTED";
+        case TG_ERR_CUDA: return "TG_ERR_CUDA";
+        case TG_ERR_TIMEOUT: return "TG_ERR_TIMEOUT";
+        case TG_ERR_NO_DEVICE: return "TG_ERR_NO_DEVICE";
+    }
+    return "TG_ERR_UNKNOWN";
+}
+
+tg_status tg_last_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TG_ERR_CUDA;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, tg::g_device_status, sizeof v) != cudaSuccess) return TG_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(tg::g_device_status, &zero, sizeof zero) != cudaSuccess)
+        return TG_ERR_CUDA;
+    return static_cast<tg_status>(v);
+}
+
+int tg_num_sms(void) {
+    int dev;
+    const tg::DeviceInfo* d = tg::current_device(&dev);
+    return d ? d->num_sms : -1;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// gemm_tc.cu -- launcher for the tensor-core GEMM (fp16, bf16, TF32 mode).
+#include "gemm_tc.cuh"
+#include "host.cuh"
+#include "launch.h"
+
+namespace tg {
+
+namespace {
+
+using CfgBF16 = TcCfg<2, 1, OutT::BF16, 256, 4>;
+using CfgF16 = TcCfg<2, 0, OutT::F16, 256, 4>;
+using CfgTF32 = TcCfg<4, 2, OutT::F32, 256, 4>;
+
+template <class Cfg>
+int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, int slot) {
+    int dev = 0;
+    const DeviceInfo* di = current_device(&dev);
+    if (!di) return kNoDevice;
+    CUtensorMap tA, tB, tC;
+    // A: K-major boxes of BK (128 B) x BM rows.
+    if (!tensor_map_2d(&tA, a.A, in_t, Cfg::IN_BYTES, a.K, a.M, a.lda * Cfg::IN_BYTES,
+                       Cfg::BK, Cfg::BM, true))
+        return kCudaError;
+    // B: N-major boxes of CHUNK_N (128 B) x BK rows.
+    if (!tensor_map_2d(&tB, a.B, in_t, Cfg::IN_BYTES, a.N, a.K, a.ldb * Cfg::IN_BYTES,
+                       Cfg::CHUNK_N, Cfg::BK, true))
+        return kCudaError;
+    // C: 32-row staging boxes of CW (128 B) columns.
+    if (!tensor_map_2d(&tC, a.C, out_t, Cfg::OUT_BYTES, a.N, a.M, a.ldc * Cfg::OUT_BYTES,
+                       Cfg::CW, 32, true))
+        return kCudaError;
+    auto kern = tc_gemm_kernel<Cfg>;
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return kCudaError;
+    const long long ntm = (a.M + Cfg::BM - 1) / Cfg::BM;
+    const long long ntn = (a.N + Cfg::BN - 1) / Cfg::BN;
+    const long long tiles = ntm * ntn;
+    const int grid = static_cast<int>(tiles < di->num_sms ? tiles : di->num_sms);
+    TcParams p;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.relu = a.relu;
+    p.inject = inject_mode();
+    p.timeout_ns = wait_limit_ns();
+    p.status = device_status_ptr();
+    if (!p.status) return kCudaError;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, tC, p);
+    return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
+}
+
+}  // namespace
+
+int launch_tc_bf16(const GemmArgs& a) {
+    return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
+}
+int launch_tc_f16(const GemmArgs& a) {
+    return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
+}
+int launch_tc_tf32(const GemmArgs& a) {
+    return run<CfgTF32>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2);
+}
+
+}  // namespace tg

@@ -1,0 +1,38 @@
+// host.cuh -- host-side helpers shared by the launchers: device facts,
+// tensor-map (TMA descriptor) encoding with a cache, debug knobs.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tg {
+
+struct DeviceInfo {
+    int ok;            // 1 if an sm_100 device
+    int num_sms;
+};
+
+// Facts about the current device (cached per device).  Returns nullptr if
+// no device is current or it is not sm_100.
+const DeviceInfo* current_device(int* dev_out);
+
+// Encode (or fetch from the cache) a 2-D tiled tensor map over a row-major
+// matrix: `cols` x `rows` elements, row pitch `ld_bytes`, box `box_cols` x
+// `box_rows`, 128-byte swizzle if `swizzle128`.  Returns false on failure.
+bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype,
+                   int elem_bytes, uint64_t cols, uint64_t rows, uint64_t ld_bytes,
+                   uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+
+// Bounded-wait limit for kernels, in ns (TG_DEBUG_TIMEOUT_US overrides).
+unsigned long long wait_limit_ns();
+
+// Debug fault-injection selector (TG_INJECT, default 0 = off).
+int inject_mode();
+
+// Device address of the current device's status word (nullptr on error).
+int* device_status_ptr();
+
+// Allow `func` to use `bytes` of dynamic shared memory (once per device).
+cudaError_t set_smem_attr(const void* func, int bytes, int slot);
+
+}  // namespace tg

@@ -1,0 +1,29 @@
+// launch.h -- internal interface between the C ABI shim and the launchers.
+// Arguments arrive here already validated (sizes, pointers, alignment).
+#pragma once
+#include <cstdint>
+
+namespace tg {
+
+// Internal status values; identical to the tg_status codes.
+enum : int { kOk = 0, kInvalidArg = 1, kAlignment = 2, kUnsupported = 3, kCudaError = 4,
+             kTimeout = 5, kNoDevice = 6 };
+
+struct GemmArgs {
+    int64_t M, N, K;
+    const void* A; int64_t lda;      // elements
+    const void* B; int64_t ldb;      // elements (bytes for packed 4-bit weights)
+    void* C; int64_t ldc;            // elements
+    const void* scales; int64_t lds; // 4-bit path only
+    int group;                       // 4-bit path only
+    int relu;
+    void* stream;
+};
+
+int launch_tc_bf16(const GemmArgs& a);
+int launch_tc_f16(const GemmArgs& a);
+int launch_tc_tf32(const GemmArgs& a);
+int launch_ffma_f32(const GemmArgs& a);
+int launch_w4a16(const GemmArgs& a);
+
+}  // namespace tg
