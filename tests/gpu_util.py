@@ -7,14 +7,30 @@ SENTINEL32 = np.float32(-12345.678)
 
 
 def to_dev(arr, kind):
-    """numpy stored values -> CUDA tensor. kind: 'f32', 'f16', 'bf16', 'u8'."""
+    """numpy stored values -> CUDA tensor. kind: 'f32', 'f16', 'bf16', 'u8'.
+
+    The device copy's row pitch is rounded up to a multiple of 16 bytes (the
+    library requires it), so odd widths come back as strided views."""
     import torch
+    arr = np.asarray(arr)
+    rows, cols = arr.shape
+    eb = {"f32": 4, "u8": 1}.get(kind, 2)
+    per = 16 // eb
+    ld = max(per, -(-cols // per) * per)
     if kind == "f32":
-        return torch.from_numpy(np.ascontiguousarray(arr, np.float32)).cuda()
-    if kind == "u8":
-        return torch.from_numpy(np.ascontiguousarray(arr, np.uint8)).cuda()
-    t = torch.from_numpy(np.ascontiguousarray(arr, np.uint16).view(np.int16)).cuda()
-    return t.view(torch.float16 if kind == "f16" else torch.bfloat16)
+        host = np.zeros((rows, ld), np.float32)
+        host[:, :cols] = arr
+        t = torch.from_numpy(host).cuda()
+    elif kind == "u8":
+        host = np.zeros((rows, ld), np.uint8)
+        host[:, :cols] = arr
+        t = torch.from_numpy(host).cuda()
+    else:
+        host = np.zeros((rows, ld), np.uint16)
+        host[:, :cols] = arr
+        t = torch.from_numpy(host.view(np.int16)).cuda()
+        t = t.view(torch.float16 if kind == "f16" else torch.bfloat16)
+    return t[:, :cols]
 
 
 def from_dev(t, kind):

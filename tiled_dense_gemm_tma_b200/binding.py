@@ -77,11 +77,12 @@ def _stream_handle(stream):
 
 
 def _ld(t, name):
+    """Row pitch (elements) of a row-major 2-D tensor view."""
     if t.dim() != 2:
         raise ValueError(f"{name} must be 2-D")
     if t.stride(1) != 1 and t.shape[1] > 1:
         raise ValueError(f"{name} must be row-major (unit column stride)")
-    return max(t.stride(0), t.shape[1]) if t.shape[0] <= 1 else t.stride(0)
+    return t.stride(0)
 
 
 def _check(code, what):

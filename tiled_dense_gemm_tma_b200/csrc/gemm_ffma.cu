@@ -1,0 +1,207 @@
+// gemm_ffma.cu -- fp32 GEMM on the CUDA cores (exact fp32 products, fp32
+// FMA accumulation), the fp32 kernel of "TileLang ... 高效 GEMM 内核"
+// (mhpq.cn), section 3.2: 128 x 128 output tiles, BK = 32 slices along K,
+// 256 computing threads; section 3.3: slices staged in shared memory and
+// reused, loads overlapped with math, float4 vector reads.
+//
+// B200 mapping:
+//   warp 8      TMA producer: fills a STAGES-deep ring with the A slice
+//               (128 rows x 32 floats = 128 B per row, 128-byte swizzle) and
+//               the B slice (32 rows x 128 floats, unswizzled), arming full[s].
+//   warps 0-7   compute: thread (tm, tn) owns rows tm + 16 i (i < 8) and
+//               columns 4 tn + j, 64 + 4 tn + j (j < 4): an 8 x 8 register
+//               tile.  Per 4 k-steps it reads 8 float4 of A (one per row,
+//               along k) and per k-step 2 float4 of B; each float4 pair feeds
+//               64 FFMAs.  The swizzle makes the A reads of a warp (4 rows,
+//               same k chunk) hit 4 distinct bank groups.
+//   The accumulators go straight to global memory with float4 stores (a
+//   warp writes 4 rows x 128 contiguous bytes), clipped at the matrix edge.
+#include "ptx.cuh"
+#include "host.cuh"
+#include "launch.h"
+
+namespace tg {
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 32, STAGES = 4;
+constexpr int A_STAGE = BM * BK * 4;     // 16 KB
+constexpr int B_STAGE = BK * BN * 4;     // 16 KB
+constexpr int COMPUTE_WARPS = 8;
+constexpr int THREADS = 32 * (COMPUTE_WARPS + 1);
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 128 + 1024;
+
+struct FfmaParams {
+    int M, N, K, ldc;
+    int relu;
+    unsigned long long timeout_ns;
+    int* status;
+    float* C;
+};
+
+__device__ __forceinline__ float4 lds128(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                 const __grid_constant__ CUtensorMap tmB,
+                 const FfmaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + STAGES * A_STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smB + STAGES * B_STAGE);
+    uint64_t* empty = full + STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_kb = (p.K + BK - 1) / BK;
+    const int m0 = blockIdx.y * BM;
+    const int n0 = blockIdx.x * BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], COMPUTE_WARPS);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    if (warp == COMPUTE_WARPS) {
+        // ---------------------------------------------------- TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t ph = (kb / STAGES) & 1;
+                if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, p.timeout_ns, p.status)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                tma_load_2d(smA + s * A_STAGE, &tmA, &full[s], kb * BK, m0);
+                tma_load_2d(smB + s * B_STAGE, &tmB, &full[s], n0, kb * BK);
+            }
+            if (!ok) {
+                for (int s = 0; s < STAGES; ++s)
+                    if (armed & (1u << s)) {
+                        volatile int never = 0;
+                        bounded_wait(&full[s], (armed_par >> s) & 1, &never, p.timeout_ns, p.status);
+                    }
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------- compute warps
+    const int tm = (warp >> 1) * 4 + (lane >> 3);     // 0..15
+    const int tn = (warp & 1) * 8 + (lane & 7);       // 0..15
+    const uint32_t xr = static_cast<uint32_t>(tm & 7); // swizzle phase of all 8 rows
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    const uint32_t a_base0 = smem_u32(smA) + tm * 128;
+    const uint32_t b_base0 = smem_u32(smB) + tn * 16;
+    for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!bounded_wait(&full[s], ph, abort_flag, p.timeout_ns, p.status)) break;
+        const uint32_t a_base = a_base0 + s * A_STAGE;
+        const uint32_t b_base = b_base0 + s * B_STAGE;
+#pragma unroll 2
+        for (int k4 = 0; k4 < BK / 4; ++k4) {
+            float4 a[8];
+            const uint32_t a_off = ((static_cast<uint32_t>(k4) ^ xr) << 4);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] = lds128(a_base + i * 16 * 128 + a_off);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t brow = b_base + (k4 * 4 + kk) * (BN * 4);
+                const float4 b0 = lds128(brow);
+                const float4 b1 = lds128(brow + 256);
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, bv[j], acc[i][j]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (*abort_flag) return;
+
+    // ---------------------------------------------------------- epilogue
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int row = m0 + tm + 16 * i;
+        if (row >= p.M) continue;
+        float* crow = p.C + static_cast<size_t>(row) * p.ldc;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int col = n0 + h * 64 + tn * 4;
+            float v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = p.relu ? fmaxf(acc[i][h * 4 + j], 0.f) : acc[i][h * 4 + j];
+            if (col + 3 < p.N) {
+                *reinterpret_cast<float4*>(crow + col) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (col + j < p.N) crow[col + j] = v[j];
+            }
+        }
+    }
+}
+
+}  // namespace
+
+int launch_ffma_f32(const GemmArgs& a) {
+    int dev = 0;
+    if (!current_device(&dev)) return kNoDevice;
+    CUtensorMap tA, tB;
+    if (!tensor_map_2d(&tA, a.A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.K, a.M, a.lda * 4,
+                       BK, BM, SWZ_128))
+        return kCudaError;
+    if (!tensor_map_2d(&tB, a.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.N, a.K, a.ldb * 4,
+                       BN, BK, SWZ_NONE))
+        return kCudaError;
+    if (set_smem_attr(reinterpret_cast<const void*>(ffma_gemm_kernel), SMEM_BYTES, 8) != cudaSuccess)
+        return kCudaError;
+    FfmaParams p;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.ldc = static_cast<int>(a.ldc);
+    p.relu = a.relu;
+    p.timeout_ns = wait_limit_ns();
+    p.status = device_status_ptr();
+    p.C = static_cast<float*>(a.C);
+    if (!p.status) return kCudaError;
+    if (a.ldc > 0x7fffffff) return kUnsupported;
+    dim3 grid(static_cast<unsigned>((a.N + BN - 1) / BN), static_cast<unsigned>((a.M + BM - 1) / BM));
+    if (grid.y > 65535) return kUnsupported;
+    ffma_gemm_kernel<<<grid, THREADS, SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, p);
+    return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
+}
+
+}  // namespace tg

@@ -19,15 +19,15 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     CUtensorMap tA, tB, tC;
     // A: K-major boxes of BK (128 B) x BM rows.
     if (!tensor_map_2d(&tA, a.A, in_t, Cfg::IN_BYTES, a.K, a.M, a.lda * Cfg::IN_BYTES,
-                       Cfg::BK, Cfg::BM, true))
+                       Cfg::BK, Cfg::BM, SWZ_128))
         return kCudaError;
     // B: N-major boxes of CHUNK_N (128 B) x BK rows.
     if (!tensor_map_2d(&tB, a.B, in_t, Cfg::IN_BYTES, a.N, a.K, a.ldb * Cfg::IN_BYTES,
-                       Cfg::CHUNK_N, Cfg::BK, true))
+                       Cfg::CHUNK_N, Cfg::BK, Cfg::IN_BYTES == 4 ? SWZ_128_32B : SWZ_128))
         return kCudaError;
     // C: 32-row staging boxes of CW (128 B) columns.
     if (!tensor_map_2d(&tC, a.C, out_t, Cfg::OUT_BYTES, a.N, a.M, a.ldc * Cfg::OUT_BYTES,
-                       Cfg::CW, 32, true))
+                       Cfg::CW, 32, SWZ_128))
         return kCudaError;
     auto kern = tc_gemm_kernel<Cfg>;
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)

@@ -55,6 +55,9 @@ struct TcCfg {
     static constexpr int B_CHUNK = BK * 128;            // bytes of one BK x CHUNK_N box
     static constexpr int B_STAGE = (BN / CHUNK_N) * B_CHUNK;
     static constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+    // N-major B: tf32 needs the 32-byte-unit swizzle (4-row atom, 512 B).
+    static constexpr uint32_t B_LAYOUT = IN_BYTES == 4 ? 1u : 2u;
+    static constexpr uint32_t B_SBO = IN_BYTES == 4 ? 512u : 1024u;
     static constexpr int CW = 128 / OUT_BYTES;          // output columns per staging row
     static constexpr int STG_BUF = 32 * 128;            // one warp's 32-row staging box
     static constexpr int EPI_WARPS = 4;
@@ -253,9 +256,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     for (int k = 0; k < Cfg::BK / Cfg::MMA_K; ++k) {
                         // A: K-major, advance 32 bytes of K inside the swizzle row.
                         const uint64_t ad = sw128_desc(a_addr + k * 32, 16, 1024);
-                        // B: N-major, advance MMA_K rows of 128 bytes.
+                        // B: N-major, advance MMA_K rows of 128 bytes.  16-bit
+                        // data uses the 8-row swizzle atom, tf32 the 4-row one.
                         const uint64_t bd = sw128_desc(b_addr + k * Cfg::MMA_K * 128,
-                                                       Cfg::B_CHUNK, 1024);
+                                                       Cfg::B_CHUNK, Cfg::B_SBO, Cfg::B_LAYOUT);
                         if (Cfg::FMT == 2) mma_tf32(d_tmem, ad, bd, idesc, (kb | k) != 0);
                         else               mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
                     }

@@ -67,7 +67,7 @@ const DeviceInfo* current_device(int* dev_out) {
 
 bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype,
                    int elem_bytes, uint64_t cols, uint64_t rows, uint64_t ld_bytes,
-                   uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -80,7 +80,7 @@ bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype
     if (rows < 1) rows = 1;
     if (cols < 1) cols = 1;
     MapKey key{reinterpret_cast<uint64_t>(base), cols, rows, ld_bytes, box_cols, box_rows,
-               static_cast<int>(dtype), swizzle128 ? 1 : 0};
+               static_cast<int>(dtype), static_cast<int>(swz)};
     {
         std::lock_guard<std::mutex> lk(g_map_mu);
         auto it = g_maps.find(key);
@@ -94,7 +94,7 @@ bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype
     std::memset(&m, 0, sizeof m);
     CUresult r = g_encode(&m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          swz,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     (void)elem_bytes;

@@ -18,10 +18,14 @@ const DeviceInfo* current_device(int* dev_out);
 
 // Encode (or fetch from the cache) a 2-D tiled tensor map over a row-major
 // matrix: `cols` x `rows` elements, row pitch `ld_bytes`, box `box_cols` x
-// `box_rows`, 128-byte swizzle if `swizzle128`.  Returns false on failure.
+// `box_rows`, shared-memory swizzle `swz`.  Returns false on failure.
 bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype,
                    int elem_bytes, uint64_t cols, uint64_t rows, uint64_t ld_bytes,
-                   uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+constexpr CUtensorMapSwizzle SWZ_NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
+constexpr CUtensorMapSwizzle SWZ_128 = CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr CUtensorMapSwizzle SWZ_128_32B = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
 
 // Bounded-wait limit for kernels, in ns (TG_DEBUG_TIMEOUT_US overrides).
 unsigned long long wait_limit_ns();

@@ -217,17 +217,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
 //   lbo / sbo: leading / stride byte offsets (multiples of 16).
 //   K-major tiles: rows of 128 B, 8-row groups `sbo` apart (lbo unused).
-//   MN-major tiles: 128 B (one swizzle row) along M/N, 8-row K groups `sbo`
+//   MN-major tiles: 128 B (one swizzle row) along M/N, K-row groups `sbo`
 //   apart, successive 128 B wide M/N column blocks `lbo` apart.
-// Layout: start>>4 in [0,14), lbo>>4 in [16,30), sbo>>4 in [32,46),
-// descriptor version 1 at [46,48), swizzle mode 2 (128 B) at [61,64).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+//   layout: 2 = 128-byte swizzle of 16-byte units (8-row atom);
+//           1 = 128-byte swizzle of 32-byte units (4-row atom), the only
+//               MN-major layout the tensor core accepts for 32-bit (tf32) data.
+// Fields: start>>4 in [0,14), lbo>>4 in [16,30), sbo>>4 in [32,46),
+// descriptor version 1 at [46,48), layout type at [61,64).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo,
+                                               uint32_t layout = 2) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;
-    d |= 2ull << 61;
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
     return d;
 }
 
