@@ -44,6 +44,8 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
+    p.C = a.C;
+    p.ldc = a.ldc;
     if (!p.status) return kCudaError;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, tC, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;

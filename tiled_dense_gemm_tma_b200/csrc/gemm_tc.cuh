@@ -76,7 +76,33 @@ struct TcParams {
     int inject;               // debug: 1 = producer skips arming the first slot
     unsigned long long timeout_ns;
     int* status;              // device status word (ST_TIMEOUT on an expired wait)
+    void* C;                  // output base and row pitch (elements), for the ragged
+    long long ldc;            // last column chunk, which is stored without TMA
 };
+
+// Store the first `valid_bytes` (< 128) of one packed 128-byte output row
+// segment with plain global stores.  The copy engine rounds a clipped store
+// up to whole 16-byte units, so a row tail narrower than that is written here.
+template <int OUT_BYTES>
+__device__ __forceinline__ void store_row_tail(uint8_t* dst, const uint4* packed, int valid_bytes) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int b0 = j * 16;
+        if (b0 + 16 <= valid_bytes) {
+            *reinterpret_cast<uint4*>(dst + b0) = packed[j];
+        } else if (b0 < valid_bytes) {
+            const uint32_t w[4] = {packed[j].x, packed[j].y, packed[j].z, packed[j].w};
+            for (int e = 0; b0 + e * OUT_BYTES < valid_bytes; ++e) {
+                if (OUT_BYTES == 4) {
+                    *reinterpret_cast<uint32_t*>(dst + b0 + 4 * e) = w[e];
+                } else {
+                    *reinterpret_cast<uint16_t*>(dst + b0 + 2 * e) =
+                        static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+                }
+            }
+        }
+    }
+}
 
 // Map a linear tile index to (tile_m, tile_n), GROUP_M tile rows per band.
 __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int group_m,
@@ -305,6 +331,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 tmem_ld_wait();
                 uint4 packed[8];
                 pack_row_chunk<Cfg::OUT>(v, p.relu, packed);
+                if (col0 + Cfg::CW > p.N) {
+                    // ragged last chunk of the row: plain stores, one row per lane
+                    const int row = row0 + lane;
+                    if (row < p.M) {
+                        uint8_t* dst = static_cast<uint8_t*>(p.C) +
+                            (static_cast<long long>(row) * p.ldc + col0) * Cfg::OUT_BYTES;
+                        store_row_tail<Cfg::OUT_BYTES>(dst, packed, (p.N - col0) * Cfg::OUT_BYTES);
+                    }
+                    continue;
+                }
                 uint8_t* stg = stg0 + (nstore & 1) * Cfg::STG_BUF;
                 if (lane == 0) bulk_wait_read<1>();      // buffer's previous store has read it
                 __syncwarp();
