@@ -92,7 +92,9 @@ __device__ __forceinline__ void store_row_tail(uint8_t* dst, const uint4* packed
             *reinterpret_cast<uint4*>(dst + b0) = packed[j];
         } else if (b0 < valid_bytes) {
             const uint32_t w[4] = {packed[j].x, packed[j].y, packed[j].z, packed[j].w};
-            for (int e = 0; b0 + e * OUT_BYTES < valid_bytes; ++e) {
+#pragma unroll
+            for (int e = 0; e < 16 / OUT_BYTES; ++e) {
+                if (b0 + e * OUT_BYTES >= valid_bytes) break;
                 if (OUT_BYTES == 4) {
                     *reinterpret_cast<uint32_t*>(dst + b0 + 4 * e) = w[e];
                 } else {
@@ -116,56 +118,92 @@ __device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int group_m
     tn = local / gsz;
 }
 
-template <OutT O>
-__device__ __forceinline__ void pack_row_chunk(const uint32_t* v, int relu, uint4* out);
+// Source position, inside an 8-column group, of output column q when the
+// group's accumulator columns are stored in the order 0,2,4,6,1,3,5,7 (the
+// order the 4-bit weight converter produces).
+__device__ __forceinline__ constexpr int perm8_src(int q) { return (q >> 1) | ((q & 1) << 2); }
 
 // 64 fp32 accumulators -> 64 fp16 / bf16 (8 x 16 B); 32 -> 32 fp32 (8 x 16 B).
-template <>
-__device__ __forceinline__ void pack_row_chunk<OutT::BF16>(const uint32_t* v, int relu, uint4* out) {
+// PERM8: undo the 0,2,4,6,1,3,5,7 column order inside each 8-column group.
+template <OutT O, bool PERM8>
+__device__ __forceinline__ void pack_row_chunk(const uint32_t* v, int relu, uint4* out) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         uint32_t w[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-            float x0 = __uint_as_float(v[j * 8 + 2 * h]);
-            float x1 = __uint_as_float(v[j * 8 + 2 * h + 1]);
-            if (relu) { x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); }
-            __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
-            w[h] = *reinterpret_cast<uint32_t*>(&p);
+            if constexpr (O == OutT::F32) {
+                float x = __uint_as_float(v[j * 4 + h]);
+                if (relu) x = fmaxf(x, 0.f);
+                w[h] = __float_as_uint(x);
+            } else {
+                const int i0 = PERM8 ? perm8_src(2 * h) : 2 * h;
+                const int i1 = PERM8 ? perm8_src(2 * h + 1) : 2 * h + 1;
+                float x0 = __uint_as_float(v[j * 8 + i0]);
+                float x1 = __uint_as_float(v[j * 8 + i1]);
+                if (relu) { x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); }
+                if constexpr (O == OutT::BF16) {
+                    __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+                    w[h] = *reinterpret_cast<uint32_t*>(&pr);
+                } else {
+                    __half2 pr = __floats2half2_rn(x0, x1);
+                    w[h] = *reinterpret_cast<uint32_t*>(&pr);
+                }
+            }
         }
         out[j] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
-template <>
-__device__ __forceinline__ void pack_row_chunk<OutT::F16>(const uint32_t* v, int relu, uint4* out) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint32_t w[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            float x0 = __uint_as_float(v[j * 8 + 2 * h]);
-            float x1 = __uint_as_float(v[j * 8 + 2 * h + 1]);
-            if (relu) { x0 = fmaxf(x0, 0.f); x1 = fmaxf(x1, 0.f); }
-            __half2 p = __floats2half2_rn(x0, x1);
-            w[h] = *reinterpret_cast<uint32_t*>(&p);
+// Epilogue of one output tile for the 32 rows of TMEM lane quarter q:
+// tcgen05.ld the accumulator columns CW at a time, ReLU, round, write a
+// 128-byte-swizzled 32-row staging box and TMA-store it; the ragged last
+// chunk of a row (narrower than CW columns) is stored per lane instead.
+// NBUF staging buffers of 4 KB per warp rotate through `nstore`.
+template <OutT OUT, int BN, bool PERM8, int NBUF>
+__device__ __forceinline__ void epilogue_tile(const CUtensorMap* tmC, const TcParams& p,
+                                              uint32_t tmem_tile, int q, int lane,
+                                              int row0, int n0, uint8_t* stg0,
+                                              uint32_t& nstore) {
+    constexpr int OUT_BYTES = OUT == OutT::F32 ? 4 : 2;
+    constexpr int CW = 128 / OUT_BYTES;
+    constexpr int STG_BUF = 32 * 128;
+    if (row0 >= p.M) return;                               // warp-uniform
+#pragma unroll 1
+    for (int c = 0; c < BN / CW; ++c) {
+        const int col0 = n0 + c * CW;
+        if (col0 >= p.N) break;
+        const uint32_t taddr = tmem_tile + (static_cast<uint32_t>(q * 32) << 16) + c * CW;
+        uint32_t v[CW];
+        tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        if constexpr (CW == 64)
+            tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        uint4 packed[8];
+        pack_row_chunk<OUT, PERM8>(v, p.relu, packed);
+        if (col0 + CW > p.N) {
+            const int row = row0 + lane;
+            if (row < p.M) {
+                uint8_t* dst = static_cast<uint8_t*>(p.C) +
+                    (static_cast<long long>(row) * p.ldc + col0) * OUT_BYTES;
+                store_row_tail<OUT_BYTES>(dst, packed, (p.N - col0) * OUT_BYTES);
+            }
+            continue;
         }
-        out[j] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-template <>
-__device__ __forceinline__ void pack_row_chunk<OutT::F32>(const uint32_t* v, int relu, uint4* out) {
+        uint8_t* stg = stg0 + (nstore % NBUF) * STG_BUF;
+        if (lane == 0) bulk_wait_read<NBUF - 1>();         // this buffer's last store has read it
+        __syncwarp();
+        uint8_t* row = stg + lane * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint32_t w[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            float x = __uint_as_float(v[j * 4 + h]);
-            if (relu) x = fmaxf(x, 0.f);
-            w[h] = __float_as_uint(x);
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) = packed[j];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmC, stg, col0, row0);
+            bulk_commit();
         }
-        out[j] = make_uint4(w[0], w[1], w[2], w[3]);
+        ++nstore;
     }
 }
 
@@ -313,49 +351,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
             tc_fence_after();
-            const int row0 = tm * Cfg::BM + q * 32;
-            const bool rows_live = row0 < p.M;
-#pragma unroll 1
-            for (int c = 0; c < Cfg::BN / Cfg::CW; ++c) {
-                const int col0 = tn * Cfg::BN + c * Cfg::CW;
-                if (!rows_live || col0 >= p.N) continue;   // warp-uniform
-                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16)
-                                     + acc * Cfg::BN + c * Cfg::CW;
-                uint32_t v[Cfg::CW];
-                if constexpr (Cfg::CW == 64) {
-                    tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                    tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                } else {
-                    tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                }
-                tmem_ld_wait();
-                uint4 packed[8];
-                pack_row_chunk<Cfg::OUT>(v, p.relu, packed);
-                if (col0 + Cfg::CW > p.N) {
-                    // ragged last chunk of the row: plain stores, one row per lane
-                    const int row = row0 + lane;
-                    if (row < p.M) {
-                        uint8_t* dst = static_cast<uint8_t*>(p.C) +
-                            (static_cast<long long>(row) * p.ldc + col0) * Cfg::OUT_BYTES;
-                        store_row_tail<Cfg::OUT_BYTES>(dst, packed, (p.N - col0) * Cfg::OUT_BYTES);
-                    }
-                    continue;
-                }
-                uint8_t* stg = stg0 + (nstore & 1) * Cfg::STG_BUF;
-                if (lane == 0) bulk_wait_read<1>();      // buffer's previous store has read it
-                __syncwarp();
-                uint8_t* row = stg + lane * 128;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) = packed[j];
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmC, stg, col0, row0);
-                    bulk_commit();
-                }
-                ++nstore;
-            }
+            epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
+                                                       tm * Cfg::BM + q * 32, tn * Cfg::BN,
+                                                       stg0, nstore);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);

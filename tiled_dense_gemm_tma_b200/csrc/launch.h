@@ -25,5 +25,6 @@ int launch_tc_f16(const GemmArgs& a);
 int launch_tc_tf32(const GemmArgs& a);
 int launch_ffma_f32(const GemmArgs& a);
 int launch_w4a16(const GemmArgs& a);
+int launch_w4a16_large(const GemmArgs& a);
 
 }  // namespace tg
