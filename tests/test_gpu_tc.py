@@ -164,3 +164,37 @@ def test_tf32_integer_bit_exact(tg):
     assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(A, B)))
     got = _run_f32(tg, A, B, tg.F32_TF32, relu=True)
     assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(A, B, relu=True)))
+
+
+# ------------------------------------------- small M: weight-streaming kernel
+
+SKINNY = [(1, 1000, 640), (2, 384, 4096), (16, 2048, 1000), (17, 520, 333), (33, 1024, 2048),
+          (64, 130, 64), (65, 4096, 512), (100, 777, 1200), (128, 2304, 4096)]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+@pytest.mark.parametrize("shape", SKINNY)
+def test_skinny_shapes(tg, kind, shape):
+    M, N, K = shape
+    A, B = synth.normal(M, N, K, seed=3, dtype=kind, scale_by_sqrt_k=True)
+    for relu in (False, True):
+        got = decode16(_run16(tg, kind, A, B, relu), kind)
+        ref = _oracle16(kind, A, B, relu)
+        assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} relu={relu}")
+        assert rel_frob(got, ref) <= FROB[kind]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+def test_skinny_integer_bit_exact_and_repeatable(tg, kind):
+    # split-K partials are summed in a fixed order: bit-exact on integer data
+    # and identical across repeated calls on random data
+    M, N, K = 24, 1536, 256
+    A, B = synth.integers(M, N, K, seed=1, lo=-1, hi=1, dtype=kind)
+    got = _run16(tg, kind, A, B)
+    ref = _oracle16(kind, A, B)
+    rnd = oracle.round_bf16(ref) if kind == "bf16" else oracle.round_f16(ref)
+    assert np.array_equal(got, rnd)
+    A, B = synth.normal(16, 4096, 8192, seed=3, dtype=kind, scale_by_sqrt_k=True)
+    first = _run16(tg, kind, A, B)
+    for _ in range(3):
+        assert np.array_equal(_run16(tg, kind, A, B), first)

@@ -154,6 +154,10 @@ tg_status tg_last_device_status(void* stream) {
     if (cudaMemcpyFromSymbol(&v, tg::g_device_status, sizeof v) != cudaSuccess) return TG_ERR_CUDA;
     if (v != 0 && cudaMemcpyToSymbol(tg::g_device_status, &zero, sizeof zero) != cudaSuccess)
         return TG_ERR_CUDA;
+    if (v == TG_ERR_TIMEOUT) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) tg::mark_workspaces_dirty(dev);
+    }
     return static_cast<tg_status>(v);
 }
 

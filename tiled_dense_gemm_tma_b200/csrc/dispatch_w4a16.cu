@@ -1,5 +1,7 @@
 // Dispatch of the 4-bit-weight GEMM by the number of activation rows.
 #include "launch.h"
 namespace tg {
-int launch_w4a16(const GemmArgs& a) { return launch_w4a16_large(a); }
+int launch_w4a16(const GemmArgs& a) {
+    return a.M <= kSkinnyMaxM ? launch_skinny_w4a16(a) : launch_w4a16_large(a);
+}
 }

@@ -1,0 +1,375 @@
+// gemm_skinny.cuh -- weight-streaming GEMM for few activation rows (small M).
+//
+// When M is small the GEMM is bound by streaming the K x N weight matrix from
+// HBM (the skinny shapes and the small-batch dequantize GEMM).  The tile
+// scheme of the tensor-core kernel would leave most SMs idle (N/256 tiles)
+// and waste the 128-row MMA on padding rows, so this kernel swaps the
+// operands and splits the work finely:
+//
+//   D[n][m] = sum_k W[k][n] * X[m][k]        (C = D^T, X = A)
+//
+// * The weight tile (128 columns n x 64 rows k) is the MMA's 128-row operand,
+//   N-major in shared memory; the activations (MPAD >= M rows, zero-padded
+//   by the copy engine) are the MMA's N operand, K-major.  D lives in TMEM as
+//   128 lanes (n) x MPAD columns (m).
+// * Stream-K: the (tile, k-slice) units of all T = ceil(N/128) tiles are cut
+//   into G (one per SM) contiguous, equal ranges.  A CTA accumulates each
+//   maximal run of its range inside one tile (a segment).  A segment that
+//   covers a whole tile is written to C directly; otherwise its fp32 partial
+//   goes to a workspace slot and the CTA that completes the tile's last
+//   segment (counted with an atomic ticket) sums the partials in segment
+//   order -- deterministic -- applies ReLU, rounds and writes C, and resets
+//   the ticket for the next call.
+// * Weights arrive either as fp16/bf16 tiles by TMA, or as packed 4-bit
+//   weights + scales that converter warps expand (dequant.cuh).
+#pragma once
+#include "ptx.cuh"
+#include "dequant.cuh"
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace tg {
+
+enum class WKind { F16 = 0, BF16 = 1, INT4 = 2 };
+
+template <WKind W_, int MPAD_>
+struct SkCfg {
+    static constexpr WKind W = W_;
+    static constexpr int MPAD = MPAD_;                  // MMA N: 16, 32, 64 or 128
+    static constexpr int TN = 128;                      // weight columns per tile (MMA M)
+    static constexpr int BK = 64;                       // k rows per slice
+    static constexpr bool Q4 = W_ == WKind::INT4;
+    static constexpr int W_CHUNK = BK * 128;            // 64 columns x BK rows, bytes
+    static constexpr int W_BYTES = 2 * W_CHUNK;         // 16 KB fp16 weight tile
+    static constexpr int X_BYTES = MPAD * 128;          // MPAD rows x 64 fp16
+    static constexpr int Q_BYTES = Q4 ? BK * TN / 2 : 0;   // 4 KB packed
+    static constexpr int S_BYTES = Q4 ? TN * 2 : 0;        // 256 B scales
+    // ring of TMA-filled slots; for 4-bit weights a second ring of converted tiles
+    static constexpr int RAW_SLOT_USED = Q4 ? (X_BYTES + Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
+    static constexpr int RAW_SLOT = (RAW_SLOT_USED + 1023) / 1024 * 1024;   // swizzle alignment
+    static constexpr int W_STAGES = Q4 ? 4 : 0;
+    static constexpr int BUDGET = 200 * 1024 - W_STAGES * W_BYTES;
+    static constexpr int RAW_STAGES_FIT = BUDGET / RAW_SLOT;
+    static constexpr int RAW_STAGES = RAW_STAGES_FIT > 16 ? 16 : RAW_STAGES_FIT;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int CONV_WARPS = Q4 ? 8 : 0;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
+    static constexpr int TMEM_COLS = 2 * MPAD < 32 ? 32 : 2 * MPAD;
+    static constexpr int SMEM_BYTES = RAW_STAGES * RAW_SLOT + W_STAGES * W_BYTES + 512 + 1024;
+    static_assert(MPAD % 16 == 0 && MPAD <= 128, "MPAD");
+};
+
+struct SkParams {
+    int M, N, K;
+    int relu;
+    int T, KB, U;             // tiles, k-slices per tile, units = T * KB
+    int J;                    // workspace slots per tile (max segments of a tile)
+    unsigned long long timeout_ns;
+    int* status;
+    void* C;
+    long long ldc;
+    float* ws;                // [T][J][MPAD][128] fp32 partials
+    int* tickets;             // [T], zero between calls
+};
+
+// First unit of CTA c's range.
+__device__ __forceinline__ int sk_begin(int c, int U, int G) {
+    return static_cast<int>((static_cast<long long>(c) * U) / G);
+}
+
+// CTA whose range holds unit u.
+__device__ __forceinline__ int sk_owner(int u, int U, int G) {
+    int c = static_cast<int>((static_cast<long long>(u) * G) / U);
+    while (c + 1 < G && sk_begin(c + 1, U, G) <= u) ++c;
+    while (c > 0 && sk_begin(c, U, G) > u) --c;
+    return c;
+}
+
+template <WKind W>
+__device__ __forceinline__ void store_out(void* C, long long ldc, int m, int n, float v) {
+    if constexpr (W == WKind::BF16) {
+        reinterpret_cast<__nv_bfloat16*>(C)[static_cast<long long>(m) * ldc + n] = __float2bfloat16_rn(v);
+    } else {
+        reinterpret_cast<__half*>(C)[static_cast<long long>(m) * ldc + n] = __float2half_rn(v);
+    }
+}
+
+// tmW: fp16/bf16 weights (N x K view: 64-column boxes of BK rows), or the
+//      packed 4-bit weights (64-byte boxes of BK rows) for INT4;
+// tmS: scales (INT4 only); tmX: activations, K-major boxes of 64 x MPAD.
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+skinny_kernel(const __grid_constant__ CUtensorMap tmW,
+              const __grid_constant__ CUtensorMap tmS,
+              const __grid_constant__ CUtensorMap tmX,
+              const SkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint8_t* ring = smem;                                            // RAW_STAGES x RAW_SLOT
+    uint8_t* wring = ring + Cfg::RAW_STAGES * Cfg::RAW_SLOT;         // W_STAGES x W_BYTES
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wring + Cfg::W_STAGES * Cfg::W_BYTES);
+    uint64_t* full = bars;                                           // [RAW_STAGES]
+    uint64_t* rempty = full + Cfg::RAW_STAGES;                       // [RAW_STAGES]
+    uint64_t* wfull = rempty + Cfg::RAW_STAGES;                      // [W_STAGES]
+    uint64_t* wempty = wfull + Cfg::W_STAGES;                        // [W_STAGES]
+    uint64_t* tfull = wempty + Cfg::W_STAGES;                        // [2]
+    uint64_t* tempty = tfull + 2;                                    // [2]
+    uint64_t* drain = tempty + 2;
+    uint64_t* epi_bar = drain + 1;                                   // epilogue warps joined
+    uint64_t* flag_bar = epi_bar + 1;                                // ticket result published
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flag_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* last_flag = abort_flag + 1;
+
+    // slot layout: 16-bit weights [W | X]; 4-bit weights [X | Q | S]
+    auto slot_x = [&](int s) { return ring + s * Cfg::RAW_SLOT + (Cfg::Q4 ? 0 : Cfg::W_BYTES); };
+    auto slot_w = [&](int s) { return ring + s * Cfg::RAW_SLOT; };
+    auto slot_q = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::X_BYTES; };
+    auto slot_s = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::X_BYTES + Cfg::Q_BYTES; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x;
+    const int c = blockIdx.x;
+    const int u0 = sk_begin(c, p.U, G);
+    const int u1 = sk_begin(c + 1, p.U, G);
+    const int KB = p.KB;
+    const uint64_t limit = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&rempty[s], Cfg::CONV_WARPS + 1);
+        }
+        for (int s = 0; s < Cfg::W_STAGES; ++s) {
+            mbar_init(&wfull[s], Cfg::CONV_WARPS);
+            mbar_init(&wempty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], Cfg::EPI_WARPS); }
+        mbar_init(drain, 1);
+        mbar_init(epi_bar, Cfg::EPI_WARPS);
+        mbar_init(flag_bar, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmW);
+            tma_prefetch_desc(&tmX);
+            if constexpr (Cfg::Q4) tma_prefetch_desc(&tmS);
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            int it = 0;
+            for (int u = u0; u < u1; ++u, ++it) {
+                const int t = u / KB, kb = u - (u / KB) * KB;
+                const int s = it % Cfg::RAW_STAGES;
+                const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
+                if (!bounded_wait(&rempty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                if constexpr (Cfg::Q4) {
+                    mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + Cfg::Q_BYTES + Cfg::S_BYTES);
+                    tma_load_2d(slot_q(s), &tmW, &full[s], t * (Cfg::TN / 2), kb * Cfg::BK);
+                    tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::TN, (kb * Cfg::BK) / 128);
+                } else {
+                    // the second 64-column box is skipped when it starts past N
+                    const bool second = t * Cfg::TN + 64 < p.N;
+                    mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + (second ? 2 : 1) * Cfg::W_CHUNK);
+                    tma_load_2d(slot_w(s), &tmW, &full[s], t * Cfg::TN, kb * Cfg::BK);
+                    if (second)
+                        tma_load_2d(slot_w(s) + Cfg::W_CHUNK, &tmW, &full[s], t * Cfg::TN + 64,
+                                    kb * Cfg::BK);
+                }
+                tma_load_2d(slot_x(s), &tmX, &full[s], kb * Cfg::BK, 0);
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (ph << s);
+            }
+            if (!ok) {
+                for (int s = 0; s < Cfg::RAW_STAGES; ++s)
+                    if (armed & (1u << s)) {
+                        volatile int never = 0;
+                        bounded_wait(&full[s], (armed_par >> s) & 1, &never, limit, p.status);
+                    }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            constexpr uint32_t fmt = Cfg::W == WKind::BF16 ? 1u : 0u;
+            constexpr uint32_t idesc = make_idesc(fmt, Cfg::TN, Cfg::MPAD, 1, 0);
+            bool ok = true;
+            int it = 0, seg = 0;
+            uint32_t d_tmem = tmem_base;
+            for (int u = u0; u < u1 && ok; ++u, ++it) {
+                const int kb = u - (u / KB) * KB;
+                const bool first = (u == u0) || kb == 0;
+                const bool last = (u == u1 - 1) || kb == KB - 1;
+                if (first) {
+                    const uint32_t acc = seg & 1;
+                    if (!bounded_wait(&tempty[acc], ((seg >> 1) & 1) ^ 1, abort_flag, limit, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    d_tmem = tmem_base + acc * Cfg::MPAD;
+                }
+                const int s = it % Cfg::RAW_STAGES;
+                const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
+                if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) { ok = false; break; }
+                uint32_t w_addr;
+                int w = 0;
+                if constexpr (Cfg::Q4) {
+                    w = it % Cfg::W_STAGES;
+                    if (!bounded_wait(&wfull[w], (it / Cfg::W_STAGES) & 1, abort_flag, limit, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    w_addr = smem_u32(wring + w * Cfg::W_BYTES);
+                } else {
+                    w_addr = smem_u32(slot_w(s));
+                }
+                tc_fence_after();
+                const uint32_t x_addr = smem_u32(slot_x(s));
+#pragma unroll
+                for (int k = 0; k < Cfg::BK / 16; ++k) {
+                    // weights: N-major, 16 k rows of 128 B per MMA; activations: K-major
+                    const uint64_t ad = sw128_desc(w_addr + k * 16 * 128, Cfg::W_CHUNK, 1024);
+                    const uint64_t bd = sw128_desc(x_addr + k * 32, 16, 1024);
+                    mma_f16(d_tmem, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                }
+                mma_commit(&rempty[s]);
+                if constexpr (Cfg::Q4) mma_commit(&wempty[w]);
+                if (last) {
+                    mma_commit(&tfull[seg & 1]);
+                    ++seg;
+                }
+            }
+            mma_commit(drain);
+            volatile int never = 0;
+            bounded_wait(drain, 0, &never, limit, p.status);
+        }
+        __syncwarp();
+    } else if (warp < 2 + Cfg::EPI_WARPS) {
+        // --------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int etid = threadIdx.x - 64;                   // 0..127
+        const int lane_n = q * 32 + lane;                    // TMEM lane = tile-local n slot
+        // 4-bit weights are stored 0,2,4,6,1,3,5,7 inside 8-column groups
+        const int n_loc = Cfg::Q4 ? ((lane_n & ~7) | ((lane_n & 3) << 1) | ((lane_n >> 2) & 1))
+                                  : lane_n;
+        int seg = 0;
+        uint32_t nsync = 0;
+        for (int u = u0; u < u1; ++seg) {
+            const int t = u / KB;
+            const int seg_end = min(u1, (t + 1) * KB);
+            const bool whole = (u == t * KB) && (seg_end == (t + 1) * KB);
+            u = seg_end;
+            const uint32_t acc = seg & 1;
+            if (!bounded_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, limit, p.status)) break;
+            tc_fence_after();
+            const int n = t * Cfg::TN + n_loc;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::MPAD;
+            int j = 0;
+            float* slot = nullptr;
+            if (!whole) {
+                j = c - sk_owner(t * KB, p.U, G);
+                slot = p.ws + (static_cast<long long>(t) * p.J + j) * Cfg::MPAD * Cfg::TN;
+            }
+#pragma unroll 1
+            for (int mc = 0; mc < Cfg::MPAD; mc += 16) {
+                if (mc >= p.M) break;
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(taddr + mc, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = mc + i;
+                    if (m >= p.M) break;
+                    const float x = __uint_as_float(v[i]);
+                    if (whole) {
+                        if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
+                    } else {
+                        slot[m * Cfg::TN + n_loc] = x;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (whole) continue;
+            // Publish the partial, take a ticket; the tile's last contributor
+            // reduces.  The epilogue warps meet on mbarriers with bounded waits
+            // (never an unbounded bar.sync, which a warp that gave up would hang).
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_bar);
+            if (!bounded_wait(epi_bar, nsync & 1, abort_flag, limit, p.status)) break;
+            if (etid == 0) {
+                const int first = sk_owner(t * KB, p.U, G);
+                const int nseg = sk_owner(t * KB + KB - 1, p.U, G) - first + 1;
+                const int old = atomicAdd(&p.tickets[t], 1);
+                const int is_last = old == nseg - 1;
+                if (is_last) atomicExch(&p.tickets[t], 0);
+                *last_flag = is_last ? nseg : 0;
+                mbar_arrive(flag_bar);
+            }
+            if (!bounded_wait(flag_bar, nsync & 1, abort_flag, limit, p.status)) break;
+            const int nseg = *last_flag;
+            ++nsync;
+            if (nseg) {
+                __threadfence();
+                const float* base = p.ws + static_cast<long long>(t) * p.J * Cfg::MPAD * Cfg::TN;
+                for (int m = 0; m < p.M; ++m) {
+                    float sum = 0.f;
+                    for (int jj = 0; jj < nseg; ++jj)
+                        sum += __ldcg(base + (static_cast<long long>(jj) * Cfg::MPAD + m) * Cfg::TN + n_loc);
+                    if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(sum, 0.f) : sum);
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------- converters (4-bit only)
+        if constexpr (Cfg::Q4) {
+            const int ctid = threadIdx.x - 32 * (2 + Cfg::EPI_WARPS);
+            int it = 0;
+            for (int u = u0; u < u1; ++u, ++it) {
+                const int s = it % Cfg::RAW_STAGES;
+                const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
+                const int w = it % Cfg::W_STAGES;
+                const uint32_t wph = (it / Cfg::W_STAGES) & 1;
+                if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status) ||
+                    !bounded_wait(&wempty[w], wph ^ 1, abort_flag, limit, p.status))
+                    break;
+                dequant_slice<Cfg::BK, Cfg::TN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
+                    slot_q(s), slot_s(s), wring + w * Cfg::W_BYTES, ctid);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&wfull[w]);
+                    mbar_arrive(&rempty[s]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace tg

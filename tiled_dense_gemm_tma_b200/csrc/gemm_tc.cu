@@ -54,9 +54,11 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
 }  // namespace
 
 int launch_tc_bf16(const GemmArgs& a) {
+    if (a.M <= kSkinnyMaxM) return launch_skinny_bf16(a);
     return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
 }
 int launch_tc_f16(const GemmArgs& a) {
+    if (a.M <= kSkinnyMaxM) return launch_skinny_f16(a);
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
 }
 int launch_tc_tf32(const GemmArgs& a) {

@@ -26,5 +26,12 @@ int launch_tc_tf32(const GemmArgs& a);
 int launch_ffma_f32(const GemmArgs& a);
 int launch_w4a16(const GemmArgs& a);
 int launch_w4a16_large(const GemmArgs& a);
+int launch_skinny_bf16(const GemmArgs& a);
+int launch_skinny_f16(const GemmArgs& a);
+int launch_skinny_w4a16(const GemmArgs& a);
+void mark_workspaces_dirty(int dev);
+
+// Activation rows up to which the weight-streaming kernel is used.
+constexpr long long kSkinnyMaxM = 128;
 
 }  // namespace tg
