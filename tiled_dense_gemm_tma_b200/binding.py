@@ -90,6 +90,14 @@ def _check(code, what):
         raise TgError(code, what)
 
 
+def empty_out(M, N, dtype, device):
+    """An M x N output view whose row pitch is a multiple of 16 bytes."""
+    import torch
+    per = 16 // torch.tensor([], dtype=dtype).element_size()
+    ld = max(per, -(-N // per) * per)
+    return torch.empty((M, ld), dtype=dtype, device=device)[:, :N]
+
+
 def _mk(A, B, C, dtype, out_dtype):
     import torch
     M, K = A.shape
@@ -102,7 +110,7 @@ def _mk(A, B, C, dtype, out_dtype):
         if not t.is_cuda:
             raise ValueError(f"{n} must be a CUDA tensor")
     if C is None:
-        C = torch.empty((M, N), dtype=out_dtype, device=A.device)
+        C = empty_out(M, N, out_dtype, A.device)
     elif C.shape != (M, N) or C.dtype != out_dtype:
         raise ValueError("C has the wrong shape or dtype")
     return M, N, K, C
@@ -155,7 +163,7 @@ def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None
     if Bq.shape[0] != K:
         raise ValueError("Bq must have K rows")
     if C is None:
-        C = torch.empty((M, N), dtype=torch.float16, device=A.device)
+        C = empty_out(M, N, torch.float16, A.device)
     _check(lib.tg_gemm_w4a16(M, N, K, A.data_ptr(), _ld(A, "A"), Bq.data_ptr(), _ld(Bq, "Bq"),
                              scales.data_ptr(), _ld(scales, "scales"), group_size,
                              C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
