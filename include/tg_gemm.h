@@ -133,6 +133,29 @@ TG_API tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
                         void *C, int64_t ldc,
                         int epilogue, void *stream);
 
+/*
+ * tg_gemm_bf16_small_m_static -- tg_gemm_bf16 for M <= 128 that never
+ * allocates device memory.  The pages have no counterpart: this entry point
+ * exists for callers that may not call cudaMalloc / cudaFree where they run
+ * the GEMM (a memory pool that already holds the device's free memory, or a
+ * latency-critical loop that must stay out of the driver's allocator).
+ *
+ * Same arguments, semantics and alignment rules as tg_gemm_bf16; M must be
+ * <= 128 (else TG_ERR_UNSUPPORTED).  The split-K scratch of the small-M
+ * kernel lives in a fixed device array of 16 MiB of fp32 partials plus 4096
+ * tile tickets that is part of the library image; shapes needing more return
+ * TG_ERR_UNSUPPORTED.  Every call shares that array (tickets are cleared at
+ * the start of each call): calls that overlap on the GPU, e.g. on two
+ * streams, race and give wrong results -- serialise them.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress) and
+ * caches it; make that first call before any stream capture.
+ */
+TG_API tg_status tg_gemm_bf16_small_m_static(int64_t M, int64_t N, int64_t K,
+                                             const void *A, int64_t lda,
+                                             const void *B, int64_t ldb,
+                                             void *C, int64_t ldc,
+                                             int epilogue, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 TG_API const char *tg_status_string(tg_status s);
 

@@ -10,6 +10,7 @@ The binding loads ``libtg_gemm.so`` on first use and raises if it is
 missing; there is no CPU or library fallback.
 """
 from .binding import (  # noqa: F401
-    TgError, gemm_f32, gemm_f16, gemm_bf16, gemm_w4a16, last_device_status,
+    TgError, gemm_f32, gemm_f16, gemm_bf16, gemm_w4a16, gemm_bf16_small_m_static,
+    last_device_status,
     lib_path, load_library, EPI_NONE, EPI_RELU, F32_FFMA, F32_TF32,
 )

@@ -20,6 +20,7 @@ STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
 
 # Every symbol include/tg_gemm.h declares.
 EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
+           "tg_gemm_bf16_small_m_static",
            "tg_status_string", "tg_last_device_status", "tg_num_sms")
 
 _lib = None
@@ -51,12 +52,12 @@ def load_library():
         lib = ctypes.CDLL(path)
         i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
         lib.tg_gemm_f32.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, ci, vp]
-        for name in ("tg_gemm_f16", "tg_gemm_bf16"):
+        for name in ("tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_bf16_small_m_static"):
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, vp]
         lib.tg_gemm_w4a16.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
                                       vp, i64, ci, vp]
         for name in ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
-                     "tg_last_device_status"):
+                     "tg_gemm_bf16_small_m_static", "tg_last_device_status"):
             getattr(lib, name).restype = ci
         lib.tg_status_string.argtypes = [ci]
         lib.tg_status_string.restype = ctypes.c_char_p
@@ -168,6 +169,20 @@ def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None
                              scales.data_ptr(), _ld(scales, "scales"), group_size,
                              C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
                              _stream_handle(stream)), "tg_gemm_w4a16")
+    return C
+
+
+def gemm_bf16_small_m_static(A, B, C=None, relu=False, stream=None):
+    """bf16 GEMM for M <= 128 whose scratch is a fixed device array of the
+    library: the call never allocates device memory (C must then be given
+    by a caller that cannot allocate)."""
+    import torch
+    lib = load_library()
+    M, N, K, C = _mk(A, B, C, torch.bfloat16, torch.bfloat16)
+    _check(lib.tg_gemm_bf16_small_m_static(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(),
+                                           _ld(B, "B"), C.data_ptr(), _ld(C, "C"),
+                                           EPI_RELU if relu else EPI_NONE, _stream_handle(stream)),
+           "tg_gemm_bf16_small_m_static")
     return C
 
 

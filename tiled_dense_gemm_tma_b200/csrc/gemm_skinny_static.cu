@@ -1,0 +1,183 @@
+// gemm_skinny_static.cu -- tg_gemm_bf16_small_m_static: the small-M bf16 GEMM
+// (weight-streaming, stream-K kernel of gemm_skinny.cuh) with its scratch
+// memory in a fixed array of device memory that is part of the library
+// image, so a call never allocates.
+//
+// Who needs this: code that may not call cudaMalloc / cudaFree at the point
+// where it runs the GEMM -- for example a program whose memory pool has
+// already reserved the device's free memory (a new cudaMalloc there fails or
+// steals from the pool), or a latency-critical loop that must not enter the
+// driver's allocator (cudaMalloc can take milliseconds and cudaFree waits for
+// the whole device).  The regular tg_gemm_bf16 allocates its workspace once
+// per stream on first use; this entry point never does.
+//
+// Limits and sharing:
+// - Scratch: kStaticPartialFloats fp32 partials (16 MiB) and kStaticTickets
+//   (4096) tile tickets.  The CUDA runtime places the arrays in device memory
+//   of every GPU on which this part of the library is loaded (at the latest
+//   on the first call there) and keeps them until the process exits.  Shapes
+//   whose partials or tiles exceed that return TG_ERR_UNSUPPORTED.
+// - Every call uses the same array.  Tickets are cleared at the start of each
+//   call; partials are overwritten before they are read.  Calls that overlap
+//   on the GPU (different streams, or different host threads on one device)
+//   race on the array and give wrong results: serialise them.
+// - Set-up: the first call on each device looks up the array's device address
+//   with cudaGetSymbolAddress (the array's name in host code is only a host
+//   stand-in) and caches it; make that first call before any stream capture.
+#include "gemm_skinny.cuh"
+#include "host.cuh"
+#include "launch.h"
+#include "../../include/tg_gemm.h"
+
+#include <cstring>
+#include <mutex>
+
+namespace tg {
+
+namespace {
+
+constexpr long long kStaticPartialFloats = 4ll << 20;     // 16 MiB of fp32 partials
+constexpr long long kStaticTickets = 4096;
+
+static __device__ __align__(256) float g_static_partials[kStaticPartialFloats];
+static __device__ __align__(256) int g_static_tickets[kStaticTickets];
+
+constexpr int kMaxDevs = 64;
+float* g_part_ptr[kMaxDevs];
+int* g_tick_ptr[kMaxDevs];
+std::once_flag g_setup_once[kMaxDevs];
+cudaError_t g_setup_err[kMaxDevs];
+
+// Device addresses of the two arrays for device `dev` (which is current).
+bool static_scratch(int dev, float** part, int** tick) {
+    std::call_once(g_setup_once[dev], [dev] {
+        void* p = nullptr;
+        void* t = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_partials);
+        if (e == cudaSuccess) e = cudaGetSymbolAddress(&t, g_static_tickets);
+        g_setup_err[dev] = e;
+        g_part_ptr[dev] = static_cast<float*>(p);
+        g_tick_ptr[dev] = static_cast<int*>(t);
+    });
+    if (g_setup_err[dev] != cudaSuccess || !g_part_ptr[dev] || !g_tick_ptr[dev]) return false;
+    *part = g_part_ptr[dev];
+    *tick = g_tick_ptr[dev];
+    return true;
+}
+
+long long sbegin(long long c, long long U, long long G) { return c * U / G; }
+
+long long sowner(long long u, long long U, long long G) {
+    long long c = u * G / U;
+    while (c + 1 < G && sbegin(c + 1, U, G) <= u) ++c;
+    while (c > 0 && sbegin(c, U, G) > u) --c;
+    return c;
+}
+
+// A tensor map encoded directly (no cache insertion, so no host allocation).
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                             const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                             const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                             CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                uint64_t ld_bytes, uint32_t box_cols, uint32_t box_rows) {
+    static EncodeFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeFn>(nullptr);
+        return reinterpret_cast<EncodeFn>(f);
+    }();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols < 1 ? 1 : cols, rows < 1 ? 1 : rows};
+    cuuint64_t strides[1] = {ld_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    std::memset(m, 0, sizeof *m);
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <int MPAD>
+tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                     const void* B, int64_t ldb, void* C, int64_t ldc, int relu,
+                     void* stream, const DeviceInfo* di, int dev) {
+    using Cfg = SkCfg<WKind::BF16, MPAD>;
+    const long long T = (N + Cfg::TN - 1) / Cfg::TN;
+    const long long KB = (K + Cfg::BK - 1) / Cfg::BK;
+    const long long U = T * KB;
+    if (U > 0x7fffffffll) return TG_ERR_UNSUPPORTED;
+    const long long G = U < di->num_sms ? U : di->num_sms;
+    long long J = 1;
+    for (long long t = 0; t < T; ++t) {
+        const long long n = sowner(t * KB + KB - 1, U, G) - sowner(t * KB, U, G) + 1;
+        if (n > J) J = n;
+    }
+    if (T > kStaticTickets || T * J * MPAD * Cfg::TN > kStaticPartialFloats)
+        return TG_ERR_UNSUPPORTED;                     // beyond the fixed scratch size
+    float* part = nullptr;
+    int* tick = nullptr;
+    if (!static_scratch(dev, &part, &tick)) return TG_ERR_CUDA;
+    CUtensorMap tW, tX;
+    if (!encode_map(&tW, B, N, K, ldb * 2, 64, Cfg::BK)) return TG_ERR_CUDA;
+    if (!encode_map(&tX, A, K, M, lda * 2, Cfg::BK, MPAD)) return TG_ERR_CUDA;
+    auto kern = skinny_kernel<Cfg>;
+    const int slot = 40 + (MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3);
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return TG_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(tick, 0, static_cast<size_t>(T) * sizeof(int), s) != cudaSuccess)
+        return TG_ERR_CUDA;
+    SkParams p;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.relu = relu;
+    p.T = static_cast<int>(T);
+    p.KB = static_cast<int>(KB);
+    p.U = static_cast<int>(U);
+    p.J = static_cast<int>(J);
+    p.timeout_ns = wait_limit_ns();
+    p.status = device_status_ptr();
+    p.C = C;
+    p.ldc = ldc;
+    p.ws = part;
+    p.tickets = tick;
+    if (!p.status) return TG_ERR_CUDA;
+    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(tW, tW, tX, p);
+    return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+}
+
+}  // namespace
+
+}  // namespace tg
+
+extern "C" tg_status tg_gemm_bf16_small_m_static(int64_t M, int64_t N, int64_t K, const void* A,
+                                                 int64_t lda, const void* B, int64_t ldb, void* C,
+                                                 int64_t ldc, int epilogue, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
+    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return TG_OK;
+    if (M > 128) return TG_ERR_UNSUPPORTED;            // the small-M kernel's limit
+    if (!C || ldc < N || (K > 0 && (!A || !B || lda < K || ldb < N))) return TG_ERR_INVALID_ARG;
+    if (N > 0x7fffffffll || K > 0x7fffffffll) return TG_ERR_UNSUPPORTED;
+    auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!al(C) || (ldc * 2) % 16) return TG_ERR_ALIGNMENT;
+    if (K > 0 && (!al(A) || !al(B) || (lda * 2) % 16 || (ldb * 2) % 16)) return TG_ERR_ALIGNMENT;
+    int dev = 0;
+    const tg::DeviceInfo* di = tg::current_device(&dev);
+    if (!di || dev >= tg::kMaxDevs) return TG_ERR_NO_DEVICE;
+    if (K == 0)                                        // C = epi(0) = 0
+        return cudaMemset2DAsync(C, static_cast<size_t>(ldc * 2), 0, static_cast<size_t>(N * 2),
+                                 static_cast<size_t>(M), static_cast<cudaStream_t>(stream)) ==
+                       cudaSuccess ? TG_OK : TG_ERR_CUDA;
+    const int relu = epilogue == TG_EPI_RELU;
+    if (M <= 16) return tg::run_static<16>(M, N, K, A, lda, B, ldb, C, ldc, relu, stream, di, dev);
+    if (M <= 32) return tg::run_static<32>(M, N, K, A, lda, B, ldb, C, ldc, relu, stream, di, dev);
+    if (M <= 64) return tg::run_static<64>(M, N, K, A, lda, B, ldb, C, ldc, relu, stream, di, dev);
+    return tg::run_static<128>(M, N, K, A, lda, B, ldb, C, ldc, relu, stream, di, dev);
+}
