@@ -68,7 +68,7 @@ struct SkParams {
     int* status;
     void* C;
     long long ldc;
-    float* ws;                // [T][J][MPAD][128] fp32 partials
+    float* ws;                // [T][J] slots of MPAD*128 fp32: column-major partials
     int* tickets;             // [T], zero between calls
 };
 
@@ -281,11 +281,14 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             tc_fence_after();
             const int n = t * Cfg::TN + n_loc;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::MPAD;
-            int j = 0;
+            // Partials are stored n-major, MS = M rounded up to 4 values per
+            // column, so a thread writes and reads its column with float4s.
+            const int MS = (p.M + 3) & ~3;
             float* slot = nullptr;
             if (!whole) {
-                j = c - sk_owner(t * KB, p.U, G);
-                slot = p.ws + (static_cast<long long>(t) * p.J + j) * Cfg::MPAD * Cfg::TN;
+                const int j = c - sk_owner(t * KB, p.U, G);
+                slot = p.ws + (static_cast<long long>(t) * p.J + j) * Cfg::MPAD * Cfg::TN +
+                       static_cast<long long>(n_loc) * MS;
             }
 #pragma unroll 1
             for (int mc = 0; mc < Cfg::MPAD; mc += 16) {
@@ -293,16 +296,21 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 uint32_t v[16];
                 tmem_ld_32x32b_x16(taddr + mc, v);
                 tmem_ld_wait();
+                if (whole) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int m = mc + i;
-                    if (m >= p.M) break;
-                    const float x = __uint_as_float(v[i]);
-                    if (whole) {
+                    for (int i = 0; i < 16; ++i) {
+                        const int m = mc + i;
+                        if (m >= p.M) break;
+                        const float x = __uint_as_float(v[i]);
                         if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
-                    } else {
-                        slot[m * Cfg::TN + n_loc] = x;
                     }
+                } else {
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd)
+                        if (mc + 4 * qd < MS)
+                            *reinterpret_cast<float4*>(slot + mc + 4 * qd) =
+                                make_float4(__uint_as_float(v[4 * qd]), __uint_as_float(v[4 * qd + 1]),
+                                            __uint_as_float(v[4 * qd + 2]), __uint_as_float(v[4 * qd + 3]));
                 }
             }
             tc_fence_before();
@@ -329,13 +337,46 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             const int nseg = *last_flag;
             ++nsync;
             if (nseg) {
+                // Sum the tile's partials in segment order (deterministic) with
+                // up to 4 segments x 4 float4 loads in flight per thread.
                 __threadfence();
-                const float* base = p.ws + static_cast<long long>(t) * p.J * Cfg::MPAD * Cfg::TN;
-                for (int m = 0; m < p.M; ++m) {
-                    float sum = 0.f;
-                    for (int jj = 0; jj < nseg; ++jj)
-                        sum += __ldcg(base + (static_cast<long long>(jj) * Cfg::MPAD + m) * Cfg::TN + n_loc);
-                    if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(sum, 0.f) : sum);
+                const float* base = p.ws + static_cast<long long>(t) * p.J * Cfg::MPAD * Cfg::TN +
+                                    static_cast<long long>(n_loc) * MS;
+                const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::TN;
+                for (int mb = 0; mb < MS; mb += 16) {
+                    float4 accv[4];
+#pragma unroll
+                    for (int qd = 0; qd < 4; ++qd) accv[qd] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int jj = 0; jj < nseg; jj += 4) {
+                        float4 vv[4][4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+#pragma unroll
+                            for (int qd = 0; qd < 4; ++qd)
+                                vv[r][qd] = (jj + r < nseg && mb + 4 * qd < MS)
+                                    ? __ldcg(reinterpret_cast<const float4*>(base + (jj + r) * sstride + mb + 4 * qd))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+#pragma unroll
+                            for (int qd = 0; qd < 4; ++qd) {
+                                accv[qd].x += vv[r][qd].x;
+                                accv[qd].y += vv[r][qd].y;
+                                accv[qd].z += vv[r][qd].z;
+                                accv[qd].w += vv[r][qd].w;
+                            }
+                    }
+                    if (n < p.N) {
+#pragma unroll
+                        for (int qd = 0; qd < 4; ++qd) {
+                            const float o[4] = {accv[qd].x, accv[qd].y, accv[qd].z, accv[qd].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int m = mb + 4 * qd + e;
+                                if (m < p.M) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(o[e], 0.f) : o[e]);
+                            }
+                        }
+                    }
                 }
             }
         }
