@@ -11,8 +11,9 @@ Inputs are seeded synthetic matrices (tiled_dense_gemm_tma_b200.synth),
 resident in HBM before timing starts.  The headline workload is the bf16
 GEMM M = N = K = 8192 with N(0,1)/sqrt(K) entries; its inputs (256 MB) are
 larger than the 126 MB L2, so steps run back to back without an L2 flush.
-The per-dtype breakdown flushes L2 (writes a 512 MB buffer) before every
-timed launch.
+The per-dtype breakdown flushes L2 before every timed launch (writes one
+512 MB buffer, then reads another, so no dirty lines are left to write back
+during the timed launch).
 
 Prints ONE JSON line on rank 0.  With --impl reference it times the CPU
 oracle (fp64 triple loop) on a bounded sample of the same workload instead.
@@ -265,8 +266,13 @@ class ClockSampler:
                 "samples": len(rows), "reasons": reasons}
 
 
-def flush_l2(buf):
-    buf.add_(1)
+def flush_l2(bufs):
+    """Evict L2: write a buffer larger than L2, then read a second one, so the
+    lines left in L2 are clean and the timed launch pays no write-backs."""
+    wbuf, rbuf, sink = bufs
+    wbuf.add_(1)
+    torch_sum = rbuf.sum(dtype=None)
+    sink.copy_(torch_sum)
 
 
 def time_breakdown(case, iters, warmup, flush_buf):
@@ -511,7 +517,9 @@ def main():
     # -------------------------------------------------------- breakdown
     breakdown = []
     if not args.no_breakdown and ws == 1:
-        flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        flush = (torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+                 torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+                 torch.zeros((), dtype=torch.float32, device=dev))
         del case.A
         for name in BREAKDOWN:
             try:
@@ -526,7 +534,7 @@ def main():
                                   "us_median": round(med * 1e6, 2), "us_min": round(mn * 1e6, 2),
                                   "bound": c.bound, "frac": round(c.achieved(med) / c.peak, 4),
                                   "peak": round(c.peak, 1), "peak_unit": c.unit,
-                                  "status_ok": ok, "l2": "flushed before each launch"})
+                                  "status_ok": ok, "l2": "flushed (write + clean read of 512 MB) before each launch"})
                 del c
             except Exception as exc:           # report, never hide
                 breakdown.append({"workload": name, "error": str(exc)[:200]})

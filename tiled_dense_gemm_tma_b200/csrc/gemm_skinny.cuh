@@ -47,7 +47,8 @@ struct SkCfg {
     // ring of TMA-filled slots; for 4-bit weights a second ring of converted tiles
     static constexpr int RAW_SLOT_USED = Q4 ? (X_BYTES + Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
     static constexpr int RAW_SLOT = (RAW_SLOT_USED + 1023) / 1024 * 1024;   // swizzle alignment
-    static constexpr int W_STAGES = Q4 ? 4 : 0;
+    // converted tiles in flight: deep enough to cover the MMA commit round trip
+    static constexpr int W_STAGES = Q4 ? 8 : 0;
     static constexpr int BUDGET = 200 * 1024 - W_STAGES * W_BYTES;
     static constexpr int RAW_STAGES_FIT = BUDGET / RAW_SLOT;
     static constexpr int RAW_STAGES = RAW_STAGES_FIT > 16 ? 16 : RAW_STAGES_FIT;

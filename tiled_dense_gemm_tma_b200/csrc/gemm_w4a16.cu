@@ -8,11 +8,11 @@
 //               fp16, K-major, 128-byte swizzle), the packed weight box
 //               (64 rows x BN/2 bytes) and the slice's scale row (BN fp16)
 //               into a RAW_STAGES-deep ring.
-//   warps 6-9   converters: expand the packed slice into the fp16 N-major
+//   warps 6-13  converters: expand the packed slice into the fp16 N-major
 //               swizzled B tile of a B_STAGES-deep ring (dequant_slice).
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 from the A box and the
 //               converted B tile into a double-buffered TMEM accumulator;
-//               commits release the raw slot (with the converters' four
+//               commits release the raw slot (with the converters'
 //               arrivals) and the B tile.
 //   warps 2-5   epilogue, as in the tensor-core GEMM, undoing the converter's
 //               column order inside 8-column groups.
@@ -34,7 +34,7 @@ struct W4 {
     static constexpr int B_CHUNK = BK * 128;             // 8 KB: 64 columns x BK rows
     static constexpr int B_BYTES = (BN / 64) * B_CHUNK;  // 32 KB
     static constexpr int STG_BUF = 32 * 128;
-    static constexpr int EPI_WARPS = 4, CONV_WARPS = 4;
+    static constexpr int EPI_WARPS = 4, CONV_WARPS = 8;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int GROUP_M = 16;
@@ -196,7 +196,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         __syncwarp();
     } else {
         // ------------------------------------------------------- converters
-        const int ctid = threadIdx.x - 32 * (2 + W4::EPI_WARPS);    // 0..127
+        const int ctid = threadIdx.x - 32 * (2 + W4::EPI_WARPS);    // 0..255
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
