@@ -1,5 +1,6 @@
 // gemm_tc.cu -- launcher for the tensor-core GEMM (fp16, bf16, TF32 mode).
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "host.cuh"
 #include "launch.h"
 
@@ -10,6 +11,8 @@ namespace {
 using CfgBF16 = TcCfg<2, 1, OutT::BF16, 256, 4>;
 using CfgF16 = TcCfg<2, 0, OutT::F16, 256, 4>;
 using CfgTF32 = TcCfg<4, 2, OutT::F32, 256, 4>;
+using Cfg2BF16 = Tc2Cfg<1, OutT::BF16, 6>;
+using Cfg2F16 = Tc2Cfg<0, OutT::F16, 6>;
 
 template <class Cfg>
 int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, int slot) {
@@ -51,14 +54,69 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
 }
 
+// CTA-pair kernel: 256 x 256 tiles on clusters of two CTAs.  Returns
+// kUnsupported (nothing launched) if the device refuses the cluster launch.
+template <class Cfg>
+int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
+    int dev = 0;
+    const DeviceInfo* di = current_device(&dev);
+    if (!di) return kNoDevice;
+    CUtensorMap tA, tB, tC;
+    if (!tensor_map_2d(&tA, a.A, dt, 2, a.K, a.M, a.lda * 2, Cfg::BK, Cfg::BM, SWZ_128))
+        return kCudaError;
+    if (!tensor_map_2d(&tB, a.B, dt, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128))
+        return kCudaError;
+    if (!tensor_map_2d(&tC, a.C, dt, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
+        return kCudaError;
+    auto kern = tc2_gemm_kernel<Cfg>;
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return kCudaError;
+    const long long tiles = ((a.M + Cfg::PM - 1) / Cfg::PM) * ((a.N + Cfg::BN - 1) / Cfg::BN);
+    const long long pairs_max = di->num_sms / 2;
+    const int npairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
+    TcParams p;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.relu = a.relu;
+    p.inject = inject_mode();
+    p.timeout_ns = wait_limit_ns();
+    p.status = device_status_ptr();
+    p.C = a.C;
+    p.ldc = a.ldc;
+    if (!p.status) return kCudaError;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * npairs, 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = static_cast<cudaStream_t>(a.stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tA, tB, tC, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();                       // clear; caller falls back
+        return kUnsupported;
+    }
+    return kOk;
+}
+
 }  // namespace
 
 int launch_tc_bf16(const GemmArgs& a) {
     if (a.M <= kSkinnyMaxM) return launch_skinny_bf16(a);
+    const int r = run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
+    if (r != kUnsupported) return r;
     return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
 }
 int launch_tc_f16(const GemmArgs& a) {
     if (a.M <= kSkinnyMaxM) return launch_skinny_f16(a);
+    const int r = run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
+    if (r != kUnsupported) return r;
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
 }
 int launch_tc_tf32(const GemmArgs& a) {

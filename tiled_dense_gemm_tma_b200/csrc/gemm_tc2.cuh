@@ -1,0 +1,224 @@
+// gemm_tc2.cuh -- the fp16 / bf16 GEMM on CTA pairs (tcgen05 cta_group::2).
+//
+// Same warp roles as gemm_tc.cuh, but two CTAs on neighbouring SMs (a
+// cluster of 2) share one 256 x 256 output tile: CTA rank r owns rows
+// [128 r, 128 r + 128) of the tile and stages its own A rows and its own half
+// of the tile's B columns ([128 r, 128 r + 128)).  The leader (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, N = 256: the tensor cores of both
+// SMs read A from their own CTA and B from both, and each CTA's TMEM receives
+// its 128 rows x 256 columns.  Per MMA each SM reads 4 KB of A and 4 KB of B
+// from its shared memory instead of 4 KB + 8 KB in the single-CTA kernel,
+// which relieves the shared-memory -> tensor-core path.
+//
+// Synchronisation across the pair:
+//   full[s]   leader only; both producers arm it (count 2) with their own byte
+//             counts, and both CTAs' TMA loads complete on it (.cta_group::2).
+//   empty[s]  in each CTA; the leader's MMA commit arrives on both.
+//   tfull[a]  in each CTA; the leader's MMA commit arrives on both.
+//   tempty[a] leader only; all 8 epilogue warps of the pair arrive (count 8).
+// Loads are plain tiled TMA copies: each CTA reads only its own tiles into
+// its own shared memory.  Every wait is bounded; the CTAs meet on a cluster
+// barrier after set-up and before freeing TMEM.
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace tg {
+
+template <int FMT_, OutT OUT_, int STAGES_>
+struct Tc2Cfg {
+    static constexpr int FMT = FMT_;
+    static constexpr OutT OUT = OUT_;
+    static constexpr int OUT_BYTES = 2;
+    static constexpr int BM = 128;                      // rows per CTA
+    static constexpr int PM = 256;                      // rows per pair tile
+    static constexpr int BN = 256;                      // columns per pair tile
+    static constexpr int HN = 128;                      // B columns staged per CTA
+    static constexpr int BK = 64;
+    static constexpr int MMA_K = 16;
+    static constexpr int STAGES = STAGES_;
+    static constexpr int A_STAGE = BM * 128;            // 16 KB
+    static constexpr int B_CHUNK = BK * 128;            // 8 KB: 64 columns x 64 rows
+    static constexpr int B_STAGE = (HN / 64) * B_CHUNK; // 16 KB
+    static constexpr int STG_BUF = 32 * 128;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int TMEM_COLS = 2 * BN;            // 512: double-buffered accumulator
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int GROUP_M = 8;                   // pair-tile rows per raster band
+    static constexpr int SMEM_DATA = STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * 2 * STG_BUF;
+    static constexpr int SMEM_BYTES = SMEM_DATA + 256 + 1024;
+};
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC,
+                const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + Cfg::STAGES * Cfg::A_STAGE;
+    uint8_t* smStg = smB + Cfg::STAGES * Cfg::B_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smStg + Cfg::EPI_WARPS * 2 * Cfg::STG_BUF);
+    uint64_t* full = bars;
+    uint64_t* empty = full + Cfg::STAGES;
+    uint64_t* tfull = empty + Cfg::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int ntm = (p.M + Cfg::PM - 1) / Cfg::PM;
+    const int ntn = (p.N + Cfg::BN - 1) / Cfg::BN;
+    const int num_tiles = ntm * ntn;
+    const int num_kb = (p.K + Cfg::BK - 1) / Cfg::BK;
+    const uint64_t limit = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2 * Cfg::EPI_WARPS); }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();          // peer barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both)
+        if (elect_one()) {
+            uint32_t armed = 0, armed_par = 0, it = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
+                int tm, tn;
+                tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+                const int m0 = tm * Cfg::PM + rank * Cfg::BM;
+                const int n0 = tn * Cfg::BN + rank * Cfg::HN;
+                // boxes entirely past the matrix edge are not loaded: they only
+                // feed output rows / columns that are never stored
+                const bool a_live = m0 < p.M;
+                const int b_live = n0 >= p.N ? 0 : (n0 + 64 < p.N ? 2 : 1);
+                const uint32_t bytes = (a_live ? Cfg::A_STAGE : 0) + b_live * Cfg::B_CHUNK;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const uint32_t s = it % Cfg::STAGES;
+                    const uint32_t ph = (it / Cfg::STAGES) & 1;
+                    if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                    if (p.inject == 1 && it == 0 && rank == 0) continue;   // debug: never arm slot 0
+                    const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+                    mbar_arrive_expect_tx_cluster(fbar, bytes);
+                    armed |= 1u << s;
+                    armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                    if (a_live)
+                        tma_load_2d_pair(smA + s * Cfg::A_STAGE, &tmA, fbar, kb * Cfg::BK, m0);
+                    for (int j = 0; j < b_live; ++j)
+                        tma_load_2d_pair(smB + s * Cfg::B_STAGE + j * Cfg::B_CHUNK, &tmB, fbar,
+                                         n0 + 64 * j, kb * Cfg::BK);
+                }
+            }
+            if (!ok) {
+                if (rank == 0) {
+                    for (int s = 0; s < Cfg::STAGES; ++s)
+                        if (armed & (1u << s)) {
+                            volatile int never = 0;
+                            bounded_wait(&full[s], (armed_par >> s) & 1, &never, limit, p.status);
+                        }
+                } else {
+                    // this CTA's copies complete on the leader's barriers, which it
+                    // cannot wait on: give copies in flight a fixed 1 ms to land
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 1000000ull) __nanosleep(10000);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------ MMA issuer (leader only)
+        if (rank == 0 && elect_one()) {
+            constexpr uint32_t idesc = make_idesc(Cfg::FMT, Cfg::PM, Cfg::BN, 0, 1);
+            uint32_t it = 0, tl = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs, ++tl) {
+                const uint32_t acc = tl & 1;
+                const uint32_t aph = (tl >> 1) & 1;
+                if (!bounded_wait(&tempty[acc], aph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const uint32_t s = it % Cfg::STAGES;
+                    const uint32_t ph = (it / Cfg::STAGES) & 1;
+                    if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smA + s * Cfg::A_STAGE);
+                    const uint32_t b_addr = smem_u32(smB + s * Cfg::B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < Cfg::BK / Cfg::MMA_K; ++k) {
+                        const uint64_t ad = sw128_desc(a_addr + k * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, 1024);
+                        mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+                    }
+                    const uint32_t e_loc = smem_u32(&empty[s]);
+                    mma_commit_pair(mapa_shared(e_loc, 0));      // both CTAs' slots
+                    mma_commit_pair(mapa_shared(e_loc, 1));
+                }
+                if (!ok) break;
+                const uint32_t f_loc = smem_u32(&tfull[acc]);
+                mma_commit_pair(mapa_shared(f_loc, 0));          // both CTAs' accumulators
+                mma_commit_pair(mapa_shared(f_loc, 1));
+            }
+            mma_commit_pair(mapa_shared(smem_u32(drain), 0));
+            volatile int never = 0;
+            bounded_wait(drain, 0, &never, limit, p.status);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- epilogue (both)
+        const int q = warp & 3;
+        uint8_t* stg0 = smStg + (warp - 2) * 2 * Cfg::STG_BUF;
+        uint32_t tl = 0, nstore = 0;
+        for (int t = pair; t < num_tiles; t += npairs, ++tl) {
+            int tm, tn;
+            tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+            const uint32_t acc = tl & 1;
+            const uint32_t aph = (tl >> 1) & 1;
+            if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
+            tc_fence_after();
+            epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
+                                                       tm * Cfg::PM + rank * Cfg::BM + q * 32,
+                                                       tn * Cfg::BN, stg0, nstore);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();          // the pair is done with each other's barriers and TMEM
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace tg
