@@ -55,20 +55,26 @@ __device__ __forceinline__ void scale_pairs(const uint4 s, uint32_t (&sp)[4]) {
 }
 
 // Convert a BK x BN weight slice.
-//   raw:  BK rows of BN/2 packed bytes, row pitch BN/2 (shared memory)
+//   raw:  BK rows of BN/2 packed bytes, row pitch BN/2, stored by the copy
+//         engine with its 128-byte (BN = 256) or 64-byte (BN = 128) swizzle:
+//         16-byte unit c of row k sits at unit c ^ (k & 7), resp. c ^ ((k >> 1) & 3)
 //   srow: BN fp16 scales of the slice's group (shared memory)
 //   dst:  BN/64 column blocks, CHUNK_BYTES apart; in each, row k of 64 fp16
 //         at k * 128, 16-byte unit u at ((u ^ (k & 7)) * 16) -- the N-major
 //         128-byte-swizzled operand layout.
-// NT threads share the work; `tid` in [0, NT).
+// NT threads share the work; `tid` in [0, NT).  Each group of 8 consecutive
+// threads takes 8 consecutive rows of one 32-column segment, so both its
+// swizzled reads and its swizzled writes fall in 8 distinct bank groups.
 template <int BK, int BN, int NT, int CHUNK_BYTES>
 __device__ __forceinline__ void dequant_slice(const uint8_t* raw, const uint8_t* srow,
                                               uint8_t* dst, int tid) {
+    constexpr int PITCH = BN / 2;                 // raw bytes per row: 128 or 64
     constexpr int SEGS = BN / 32;                 // 16 raw bytes = 32 columns per segment
     constexpr int ROWS_PER_PASS = NT / SEGS;
-    static_assert(NT % SEGS == 0 && BK % ROWS_PER_PASS == 0, "bad split");
-    const int seg = tid % SEGS;
-    const int r0 = tid / SEGS;
+    static_assert(BN == 256 || BN == 128, "raw row must be one swizzle span");
+    static_assert(NT % (8 * SEGS) == 0 && BK % ROWS_PER_PASS == 0, "bad split");
+    const int seg = (tid >> 3) % SEGS;
+    const int r0 = (tid & 7) + 8 * (tid / (8 * SEGS));
     uint32_t sp[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -78,7 +84,8 @@ __device__ __forceinline__ void dequant_slice(const uint8_t* raw, const uint8_t*
 #pragma unroll
     for (int i = 0; i < BK / ROWS_PER_PASS; ++i) {
         const int k = r0 + i * ROWS_PER_PASS;
-        const uint4 w = *reinterpret_cast<const uint4*>(raw + k * (BN / 2) + seg * 16);
+        const int ru = PITCH == 128 ? (seg ^ (k & 7)) : (seg ^ ((k >> 1) & 3));
+        const uint4 w = *reinterpret_cast<const uint4*>(raw + k * PITCH + (ru << 4));
         uint8_t* rowp = cbase + k * 128;
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll

@@ -78,7 +78,7 @@ int run(const GemmArgs& a) {
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
-    const long long T = (a.N + Cfg::TN - 1) / Cfg::TN;
+    const long long T = (a.N + Cfg::GN - 1) / Cfg::GN;
     const long long KB = (a.K + Cfg::BK - 1) / Cfg::BK;
     const long long U = T * KB;
     if (U > 0x7fffffffll) return kUnsupported;
@@ -90,16 +90,16 @@ int run(const GemmArgs& a) {
     }
     int* tickets = nullptr;
     float* ws = nullptr;
-    if (!get_workspace(dev, a.stream, T, T * J * MPAD * Cfg::TN * 4, &tickets, &ws))
+    if (!get_workspace(dev, a.stream, T, T * J * MPAD * Cfg::GN * 4, &tickets, &ws))
         return kCudaError;
 
     CUtensorMap tW, tS, tX;
     if constexpr (Cfg::Q4) {
         if (!tensor_map_2d(&tW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
-                           Cfg::TN / 2, Cfg::BK, SWZ_NONE))
+                           Cfg::GN / 2, Cfg::BK, SWZ_128))
             return kCudaError;
         if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
-                           a.lds * 2, Cfg::TN, 1, SWZ_NONE))
+                           a.lds * 2, Cfg::GN, 1, SWZ_NONE))
             return kCudaError;
     } else {
         const CUtensorMapDataType dt = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16

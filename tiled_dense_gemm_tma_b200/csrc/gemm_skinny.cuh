@@ -36,26 +36,30 @@ template <WKind W_, int MPAD_>
 struct SkCfg {
     static constexpr WKind W = W_;
     static constexpr int MPAD = MPAD_;                  // MMA N: 16, 32, 64 or 128
-    static constexpr int TN = 128;                      // weight columns per tile (MMA M)
+    static constexpr int TN = 128;                      // weight columns per MMA (MMA M)
     static constexpr int BK = 64;                       // k rows per slice
     static constexpr bool Q4 = W_ == WKind::INT4;
+    // 4-bit units span two 128-column sub-tiles so packed rows arrive as
+    // 128-byte runs (narrower rows stream markedly slower from HBM)
+    static constexpr int NSUB = Q4 ? 2 : 1;
+    static constexpr int GN = NSUB * TN;                // weight columns per unit
     static constexpr int W_CHUNK = BK * 128;            // 64 columns x BK rows, bytes
-    static constexpr int W_BYTES = 2 * W_CHUNK;         // 16 KB fp16 weight tile
+    static constexpr int W_BYTES = NSUB * 2 * W_CHUNK;  // fp16 weight tile of one unit
     static constexpr int X_BYTES = MPAD * 128;          // MPAD rows x 64 fp16
-    static constexpr int Q_BYTES = Q4 ? BK * TN / 2 : 0;   // 4 KB packed
-    static constexpr int S_BYTES = Q4 ? TN * 2 : 0;        // 256 B scales
+    static constexpr int Q_BYTES = Q4 ? BK * GN / 2 : 0;   // 8 KB packed
+    static constexpr int S_BYTES = Q4 ? GN * 2 : 0;        // 512 B scales
     // ring of TMA-filled slots; for 4-bit weights a second ring of converted tiles
     static constexpr int RAW_SLOT_USED = Q4 ? (X_BYTES + Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
     static constexpr int RAW_SLOT = (RAW_SLOT_USED + 1023) / 1024 * 1024;   // swizzle alignment
     // converted tiles in flight: deep enough to cover the MMA commit round trip
-    static constexpr int W_STAGES = Q4 ? 8 : 0;
+    static constexpr int W_STAGES = Q4 ? 4 : 0;
     static constexpr int BUDGET = 200 * 1024 - W_STAGES * W_BYTES;
     static constexpr int RAW_STAGES_FIT = BUDGET / RAW_SLOT;
     static constexpr int RAW_STAGES = RAW_STAGES_FIT > 16 ? 16 : RAW_STAGES_FIT;
     static constexpr int EPI_WARPS = 4;
     static constexpr int CONV_WARPS = Q4 ? 8 : 0;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
-    static constexpr int TMEM_COLS = 2 * MPAD < 32 ? 32 : 2 * MPAD;
+    static constexpr int TMEM_COLS = 2 * NSUB * MPAD < 32 ? 32 : 2 * NSUB * MPAD;
     static constexpr int SMEM_BYTES = RAW_STAGES * RAW_SLOT + W_STAGES * W_BYTES + 512 + 1024;
     static_assert(MPAD % 16 == 0 && MPAD <= 128, "MPAD");
 };
@@ -63,13 +67,13 @@ struct SkCfg {
 struct SkParams {
     int M, N, K;
     int relu;
-    int T, KB, U;             // tiles, k-slices per tile, units = T * KB
+    int T, KB, U;             // column groups (GN wide), k-slices per group, units = T * KB
     int J;                    // workspace slots per tile (max segments of a tile)
     unsigned long long timeout_ns;
     int* status;
     void* C;
     long long ldc;
-    float* ws;                // [T][J] slots of MPAD*128 fp32: column-major partials
+    float* ws;                // [T][J] slots of MPAD*GN fp32: column-major partials
     int* tickets;             // [T], zero between calls
 };
 
@@ -181,8 +185,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 if (!bounded_wait(&rempty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
                 if constexpr (Cfg::Q4) {
                     mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + Cfg::Q_BYTES + Cfg::S_BYTES);
-                    tma_load_2d(slot_q(s), &tmW, &full[s], t * (Cfg::TN / 2), kb * Cfg::BK);
-                    tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::TN, (kb * Cfg::BK) / 128);
+                    tma_load_2d(slot_q(s), &tmW, &full[s], t * (Cfg::GN / 2), kb * Cfg::BK);
+                    tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::GN, (kb * Cfg::BK) / 128);
                 } else {
                     // the second 64-column box is skipped when it starts past N
                     const bool second = t * Cfg::TN + 64 < p.N;
@@ -224,7 +228,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         break;
                     }
                     tc_fence_after();
-                    d_tmem = tmem_base + acc * Cfg::MPAD;
+                    d_tmem = tmem_base + acc * Cfg::NSUB * Cfg::MPAD;
                 }
                 const int s = it % Cfg::RAW_STAGES;
                 const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
@@ -244,11 +248,15 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 tc_fence_after();
                 const uint32_t x_addr = smem_u32(slot_x(s));
 #pragma unroll
-                for (int k = 0; k < Cfg::BK / 16; ++k) {
-                    // weights: N-major, 16 k rows of 128 B per MMA; activations: K-major
-                    const uint64_t ad = sw128_desc(w_addr + k * 16 * 128, Cfg::W_CHUNK, 1024);
-                    const uint64_t bd = sw128_desc(x_addr + k * 32, 16, 1024);
-                    mma_f16(d_tmem, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                for (int j = 0; j < Cfg::NSUB; ++j) {
+#pragma unroll
+                    for (int k = 0; k < Cfg::BK / 16; ++k) {
+                        // weights: N-major, 16 k rows of 128 B per MMA; activations: K-major
+                        const uint64_t ad = sw128_desc(w_addr + j * 2 * Cfg::W_CHUNK + k * 16 * 128,
+                                                       Cfg::W_CHUNK, 1024);
+                        const uint64_t bd = sw128_desc(x_addr + k * 32, 16, 1024);
+                        mma_f16(d_tmem + j * Cfg::MPAD, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                    }
                 }
                 mma_commit(&rempty[s]);
                 if constexpr (Cfg::Q4) mma_commit(&wempty[w]);
@@ -280,38 +288,44 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             const uint32_t acc = seg & 1;
             if (!bounded_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, limit, p.status)) break;
             tc_fence_after();
-            const int n = t * Cfg::TN + n_loc;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::MPAD;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   acc * Cfg::NSUB * Cfg::MPAD;
             // Partials are stored n-major, MS = M rounded up to 4 values per
-            // column, so a thread writes and reads its column with float4s.
+            // column, so a thread writes and reads its columns with float4s.
             const int MS = (p.M + 3) & ~3;
+            const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::GN;
             float* slot = nullptr;
             if (!whole) {
-                const int j = c - sk_owner(t * KB, p.U, G);
-                slot = p.ws + (static_cast<long long>(t) * p.J + j) * Cfg::MPAD * Cfg::TN +
-                       static_cast<long long>(n_loc) * MS;
+                const int jseg = c - sk_owner(t * KB, p.U, G);
+                slot = p.ws + (static_cast<long long>(t) * p.J + jseg) * sstride;
             }
+#pragma unroll
+            for (int j = 0; j < Cfg::NSUB; ++j) {
+                const int nj = j * Cfg::TN + n_loc;              // column within the unit
+                const int n = t * Cfg::GN + nj;
 #pragma unroll 1
-            for (int mc = 0; mc < Cfg::MPAD; mc += 16) {
-                if (mc >= p.M) break;
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(taddr + mc, v);
-                tmem_ld_wait();
-                if (whole) {
+                for (int mc = 0; mc < Cfg::MPAD; mc += 16) {
+                    if (mc >= p.M) break;
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(taddr + j * Cfg::MPAD + mc, v);
+                    tmem_ld_wait();
+                    if (whole) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int m = mc + i;
-                        if (m >= p.M) break;
-                        const float x = __uint_as_float(v[i]);
-                        if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
+                        for (int i = 0; i < 16; ++i) {
+                            const int m = mc + i;
+                            if (m >= p.M) break;
+                            const float x = __uint_as_float(v[i]);
+                            if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
+                        }
+                    } else {
+                        float* col = slot + static_cast<long long>(nj) * MS;
+#pragma unroll
+                        for (int qd = 0; qd < 4; ++qd)
+                            if (mc + 4 * qd < MS)
+                                *reinterpret_cast<float4*>(col + mc + 4 * qd) =
+                                    make_float4(__uint_as_float(v[4 * qd]), __uint_as_float(v[4 * qd + 1]),
+                                                __uint_as_float(v[4 * qd + 2]), __uint_as_float(v[4 * qd + 3]));
                     }
-                } else {
-#pragma unroll
-                    for (int qd = 0; qd < 4; ++qd)
-                        if (mc + 4 * qd < MS)
-                            *reinterpret_cast<float4*>(slot + mc + 4 * qd) =
-                                make_float4(__uint_as_float(v[4 * qd]), __uint_as_float(v[4 * qd + 1]),
-                                            __uint_as_float(v[4 * qd + 2]), __uint_as_float(v[4 * qd + 3]));
                 }
             }
             tc_fence_before();
@@ -341,9 +355,12 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 // Sum the tile's partials in segment order (deterministic) with
                 // up to 4 segments x 4 float4 loads in flight per thread.
                 __threadfence();
-                const float* base = p.ws + static_cast<long long>(t) * p.J * Cfg::MPAD * Cfg::TN +
-                                    static_cast<long long>(n_loc) * MS;
-                const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::TN;
+                const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::GN;
+                for (int j = 0; j < Cfg::NSUB; ++j) {
+                const int nj = j * Cfg::TN + n_loc;
+                const int n = t * Cfg::GN + nj;
+                const float* base = p.ws + static_cast<long long>(t) * p.J * sstride +
+                                    static_cast<long long>(nj) * MS;
                 for (int mb = 0; mb < MS; mb += 16) {
                     float4 accv[4];
 #pragma unroll
@@ -379,6 +396,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         }
                     }
                 }
+                }
             }
         }
     } else {
@@ -394,7 +412,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status) ||
                     !bounded_wait(&wempty[w], wph ^ 1, abort_flag, limit, p.status))
                     break;
-                dequant_slice<Cfg::BK, Cfg::TN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
+                dequant_slice<Cfg::BK, Cfg::GN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
                     slot_q(s), slot_s(s), wring + w * Cfg::W_BYTES, ctid);
                 fence_proxy_async_smem();
                 __syncwarp();

@@ -107,7 +107,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
                      const void* B, int64_t ldb, void* C, int64_t ldc, int relu,
                      void* stream, const DeviceInfo* di, int dev) {
     using Cfg = SkCfg<WKind::BF16, MPAD>;
-    const long long T = (N + Cfg::TN - 1) / Cfg::TN;
+    const long long T = (N + Cfg::GN - 1) / Cfg::GN;
     const long long KB = (K + Cfg::BK - 1) / Cfg::BK;
     const long long U = T * KB;
     if (U > 0x7fffffffll) return TG_ERR_UNSUPPORTED;
@@ -117,7 +117,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
         const long long n = sowner(t * KB + KB - 1, U, G) - sowner(t * KB, U, G) + 1;
         if (n > J) J = n;
     }
-    if (T > kStaticTickets || T * J * MPAD * Cfg::TN > kStaticPartialFloats)
+    if (T > kStaticTickets || T * J * MPAD * Cfg::GN > kStaticPartialFloats)
         return TG_ERR_UNSUPPORTED;                     // beyond the fixed scratch size
     float* part = nullptr;
     int* tick = nullptr;

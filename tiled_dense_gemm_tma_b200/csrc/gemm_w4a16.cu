@@ -238,7 +238,7 @@ int launch_w4a16_large(const GemmArgs& a) {
                        W4::BK, W4::BM, SWZ_128))
         return kCudaError;
     if (!tensor_map_2d(&tQ, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
-                       W4::BN / 2, W4::BK, SWZ_NONE))
+                       W4::BN / 2, W4::BK, SWZ_128))
         return kCudaError;
     if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
                        a.lds * 2, W4::BN, 1, SWZ_NONE))

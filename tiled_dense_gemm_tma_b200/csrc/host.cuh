@@ -24,6 +24,7 @@ bool tensor_map_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype
                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 
 constexpr CUtensorMapSwizzle SWZ_NONE = CU_TENSOR_MAP_SWIZZLE_NONE;
+constexpr CUtensorMapSwizzle SWZ_64 = CU_TENSOR_MAP_SWIZZLE_64B;
 constexpr CUtensorMapSwizzle SWZ_128 = CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr CUtensorMapSwizzle SWZ_128_32B = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
 
