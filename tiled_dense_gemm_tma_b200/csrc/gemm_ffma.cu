@@ -12,7 +12,7 @@
 //               columns 4 tn + j, 64 + 4 tn + j (j < 4): an 8 x 8 register
 //               tile.  Per 4 k-steps it reads 8 float4 of A (one per row,
 //               along k) and per k-step 2 float4 of B; each float4 pair feeds
-//               64 FFMAs.  The swizzle makes the A reads of a warp (4 rows,
+//               64 fp32 FMAs, issued as 32 paired FMAs (fma.rn.f32x2).  The swizzle makes the A reads of a warp (4 rows,
 //               same k chunk) hit 4 distinct bank groups.
 //   The accumulators go straight to global memory with float4 stores (a
 //   warp writes 4 rows x 128 contiguous bytes), clipped at the matrix edge.
@@ -111,11 +111,15 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int tm = (warp >> 1) * 4 + (lane >> 3);     // 0..15
     const int tn = (warp & 1) * 8 + (lane & 7);       // 0..15
     const uint32_t xr = static_cast<uint32_t>(tm & 7); // swizzle phase of all 8 rows
-    float acc[8][8];
+    // Accumulators are register pairs acc2[i][jp] = (C[i][2 jp], C[i][2 jp + 1])
+    // updated with the paired fp32 FMA (fma.rn.f32x2): each instruction does
+    // two independent fp32 FMAs, rounded exactly as two scalar FFMAs, and
+    // halves the issue slots the math needs.
+    uint64_t acc2[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+        for (int j = 0; j < 4; ++j) acc2[i][j] = 0ull;
 
     const uint32_t a_base0 = smem_u32(smA) + tm * 128;
     const uint32_t b_base0 = smem_u32(smB) + tn * 16;
@@ -134,14 +138,17 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t brow = b_base + (k4 * 4 + kk) * (BN * 4);
-                const float4 b0 = lds128(brow);
-                const float4 b1 = lds128(brow + 256);
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                uint64_t bp[4];        // (B[k][2j], B[k][2j+1]) for the thread's 8 columns
+                asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[0]), "=l"(bp[1]) : "r"(brow));
+                asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[2]), "=l"(bp[3]) : "r"(brow + 256));
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
+                    uint64_t aa;
+                    asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(av));
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av, bv[j], acc[i][j]);
+                    for (int j = 0; j < 4; ++j)
+                        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2[i][j]) : "l"(aa), "l"(bp[j]));
                 }
             }
         }
@@ -149,6 +156,12 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (lane == 0) mbar_arrive(&empty[s]);
     }
     if (*abort_flag) return;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[i][2 * j]), "=f"(acc[i][2 * j + 1]) : "l"(acc2[i][j]));
 
     // ---------------------------------------------------------- epilogue
 #pragma unroll

@@ -48,19 +48,31 @@ struct SkCfg {
     static constexpr int X_BYTES = MPAD * 128;          // MPAD rows x 64 fp16
     static constexpr int Q_BYTES = Q4 ? BK * GN / 2 : 0;   // 8 KB packed
     static constexpr int S_BYTES = Q4 ? GN * 2 : 0;        // 512 B scales
-    // ring of TMA-filled slots; for 4-bit weights a second ring of converted tiles
-    static constexpr int RAW_SLOT_USED = Q4 ? (X_BYTES + Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
+    // Ring of TMA-filled slots.  16-bit weights: [W | X], released by the MMA.
+    // 4-bit weights: [Q | S], released by the converters as soon as they have
+    // expanded it into a second ring of fp16 tiles; the activations then
+    // travel in a ring of their own, released by the MMA.
+    static constexpr int RAW_SLOT_USED = Q4 ? (Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
     static constexpr int RAW_SLOT = (RAW_SLOT_USED + 1023) / 1024 * 1024;   // swizzle alignment
-    // converted tiles in flight: deep enough to cover the MMA commit round trip
     static constexpr int W_STAGES = Q4 ? 4 : 0;
-    static constexpr int BUDGET = 200 * 1024 - W_STAGES * W_BYTES;
+    static constexpr int X_STAGES = !Q4 ? 0 : (X_BYTES * 8 <= 32 * 1024 ? 8 : (32 * 1024) / X_BYTES);
+    static constexpr int BUDGET = 212 * 1024 - W_STAGES * W_BYTES - X_STAGES * X_BYTES;
     static constexpr int RAW_STAGES_FIT = BUDGET / RAW_SLOT;
     static constexpr int RAW_STAGES = RAW_STAGES_FIT > 16 ? 16 : RAW_STAGES_FIT;
     static constexpr int EPI_WARPS = 4;
     static constexpr int CONV_WARPS = Q4 ? 8 : 0;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
-    static constexpr int TMEM_COLS = 2 * NSUB * MPAD < 32 ? 32 : 2 * NSUB * MPAD;
-    static constexpr int SMEM_BYTES = RAW_STAGES * RAW_SLOT + W_STAGES * W_BYTES + 512 + 1024;
+    // Independent accumulator sets: k-step kk of a unit accumulates into set
+    // kk % R, so consecutive small MMAs do not wait on each other's result;
+    // the epilogue adds the R sets in a fixed order.
+    static constexpr int R = (2 * NSUB * MPAD * 4 <= 512) ? 4 : (2 * NSUB * MPAD * 2 <= 512) ? 2 : 1;
+    static constexpr int ACC_COLS = R * NSUB * MPAD;          // one accumulator buffer
+    static constexpr int TMEM_USED = 2 * ACC_COLS;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 :
+                                     TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+    static_assert(TMEM_USED <= 512, "TMEM");
+    static constexpr int SMEM_BYTES = RAW_STAGES * RAW_SLOT + W_STAGES * W_BYTES +
+                                      X_STAGES * X_BYTES + 768 + 1024;
     static_assert(MPAD % 16 == 0 && MPAD <= 128, "MPAD");
 };
 
@@ -113,12 +125,15 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint8_t* ring = smem;                                            // RAW_STAGES x RAW_SLOT
     uint8_t* wring = ring + Cfg::RAW_STAGES * Cfg::RAW_SLOT;         // W_STAGES x W_BYTES
-    uint64_t* bars = reinterpret_cast<uint64_t*>(wring + Cfg::W_STAGES * Cfg::W_BYTES);
+    uint8_t* xring = wring + Cfg::W_STAGES * Cfg::W_BYTES;           // X_STAGES x X_BYTES
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xring + Cfg::X_STAGES * Cfg::X_BYTES);
     uint64_t* full = bars;                                           // [RAW_STAGES]
     uint64_t* rempty = full + Cfg::RAW_STAGES;                       // [RAW_STAGES]
     uint64_t* wfull = rempty + Cfg::RAW_STAGES;                      // [W_STAGES]
     uint64_t* wempty = wfull + Cfg::W_STAGES;                        // [W_STAGES]
-    uint64_t* tfull = wempty + Cfg::W_STAGES;                        // [2]
+    uint64_t* xfull = wempty + Cfg::W_STAGES;                        // [X_STAGES]
+    uint64_t* xempty = xfull + Cfg::X_STAGES;                        // [X_STAGES]
+    uint64_t* tfull = xempty + Cfg::X_STAGES;                        // [2]
     uint64_t* tempty = tfull + 2;                                    // [2]
     uint64_t* drain = tempty + 2;
     uint64_t* epi_bar = drain + 1;                                   // epilogue warps joined
@@ -127,11 +142,11 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;
 
-    // slot layout: 16-bit weights [W | X]; 4-bit weights [X | Q | S]
-    auto slot_x = [&](int s) { return ring + s * Cfg::RAW_SLOT + (Cfg::Q4 ? 0 : Cfg::W_BYTES); };
+    // slot layout: 16-bit weights [W | X]; 4-bit weights [Q | S] (X in xring)
+    auto slot_x = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::W_BYTES; };
     auto slot_w = [&](int s) { return ring + s * Cfg::RAW_SLOT; };
-    auto slot_q = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::X_BYTES; };
-    auto slot_s = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::X_BYTES + Cfg::Q_BYTES; };
+    auto slot_q = [&](int s) { return ring + s * Cfg::RAW_SLOT; };
+    auto slot_s = [&](int s) { return ring + s * Cfg::RAW_SLOT + Cfg::Q_BYTES; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -145,11 +160,15 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&rempty[s], Cfg::CONV_WARPS + 1);
+            mbar_init(&rempty[s], Cfg::Q4 ? Cfg::CONV_WARPS : 1);
         }
         for (int s = 0; s < Cfg::W_STAGES; ++s) {
             mbar_init(&wfull[s], Cfg::CONV_WARPS);
             mbar_init(&wempty[s], 1);
+        }
+        for (int s = 0; s < Cfg::X_STAGES; ++s) {
+            mbar_init(&xfull[s], 1);
+            mbar_init(&xempty[s], 1);
         }
         for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], Cfg::EPI_WARPS); }
         mbar_init(drain, 1);
@@ -175,7 +194,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             tma_prefetch_desc(&tmW);
             tma_prefetch_desc(&tmX);
             if constexpr (Cfg::Q4) tma_prefetch_desc(&tmS);
-            uint32_t armed = 0, armed_par = 0;
+            uint32_t armed = 0, armed_par = 0, xarmed = 0, xarmed_par = 0;
             bool ok = true;
             int it = 0;
             for (int u = u0; u < u1; ++u, ++it) {
@@ -184,9 +203,16 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
                 if (!bounded_wait(&rempty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
                 if constexpr (Cfg::Q4) {
-                    mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + Cfg::Q_BYTES + Cfg::S_BYTES);
+                    const int xs = it % Cfg::X_STAGES;
+                    const uint32_t xph = (it / Cfg::X_STAGES) & 1;
+                    if (!bounded_wait(&xempty[xs], xph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[s], Cfg::Q_BYTES + Cfg::S_BYTES);
                     tma_load_2d(slot_q(s), &tmW, &full[s], t * (Cfg::GN / 2), kb * Cfg::BK);
                     tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::GN, (kb * Cfg::BK) / 128);
+                    mbar_arrive_expect_tx(&xfull[xs], Cfg::X_BYTES);
+                    tma_load_2d(xring + xs * Cfg::X_BYTES, &tmX, &xfull[xs], kb * Cfg::BK, 0);
+                    xarmed |= 1u << xs;
+                    xarmed_par = (xarmed_par & ~(1u << xs)) | (xph << xs);
                 } else {
                     // the second 64-column box is skipped when it starts past N
                     const bool second = t * Cfg::TN + 64 < p.N;
@@ -195,8 +221,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     if (second)
                         tma_load_2d(slot_w(s) + Cfg::W_CHUNK, &tmW, &full[s], t * Cfg::TN + 64,
                                     kb * Cfg::BK);
+                    tma_load_2d(slot_x(s), &tmX, &full[s], kb * Cfg::BK, 0);
                 }
-                tma_load_2d(slot_x(s), &tmX, &full[s], kb * Cfg::BK, 0);
                 armed |= 1u << s;
                 armed_par = (armed_par & ~(1u << s)) | (ph << s);
             }
@@ -205,6 +231,11 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     if (armed & (1u << s)) {
                         volatile int never = 0;
                         bounded_wait(&full[s], (armed_par >> s) & 1, &never, limit, p.status);
+                    }
+                for (int s = 0; s < Cfg::X_STAGES; ++s)
+                    if (xarmed & (1u << s)) {
+                        volatile int never = 0;
+                        bounded_wait(&xfull[s], (xarmed_par >> s) & 1, &never, limit, p.status);
                     }
             }
         }
@@ -228,25 +259,28 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         break;
                     }
                     tc_fence_after();
-                    d_tmem = tmem_base + acc * Cfg::NSUB * Cfg::MPAD;
+                    d_tmem = tmem_base + acc * Cfg::ACC_COLS;
                 }
                 const int s = it % Cfg::RAW_STAGES;
                 const uint32_t ph = (it / Cfg::RAW_STAGES) & 1;
-                if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) { ok = false; break; }
-                uint32_t w_addr;
-                int w = 0;
+                uint32_t w_addr, x_addr;
+                int w = 0, xs = 0;
                 if constexpr (Cfg::Q4) {
                     w = it % Cfg::W_STAGES;
-                    if (!bounded_wait(&wfull[w], (it / Cfg::W_STAGES) & 1, abort_flag, limit, p.status)) {
+                    xs = it % Cfg::X_STAGES;
+                    if (!bounded_wait(&xfull[xs], (it / Cfg::X_STAGES) & 1, abort_flag, limit, p.status) ||
+                        !bounded_wait(&wfull[w], (it / Cfg::W_STAGES) & 1, abort_flag, limit, p.status)) {
                         ok = false;
                         break;
                     }
                     w_addr = smem_u32(wring + w * Cfg::W_BYTES);
+                    x_addr = smem_u32(xring + xs * Cfg::X_BYTES);
                 } else {
+                    if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) { ok = false; break; }
                     w_addr = smem_u32(slot_w(s));
+                    x_addr = smem_u32(slot_x(s));
                 }
                 tc_fence_after();
-                const uint32_t x_addr = smem_u32(slot_x(s));
 #pragma unroll
                 for (int j = 0; j < Cfg::NSUB; ++j) {
 #pragma unroll
@@ -255,11 +289,17 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         const uint64_t ad = sw128_desc(w_addr + j * 2 * Cfg::W_CHUNK + k * 16 * 128,
                                                        Cfg::W_CHUNK, 1024);
                         const uint64_t bd = sw128_desc(x_addr + k * 32, 16, 1024);
-                        mma_f16(d_tmem + j * Cfg::MPAD, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                        const int set = k % Cfg::R;
+                        mma_f16(d_tmem + (set * Cfg::NSUB + j) * Cfg::MPAD, ad, bd, idesc,
+                                (first && k < Cfg::R) ? 0u : 1u);
                     }
                 }
-                mma_commit(&rempty[s]);
-                if constexpr (Cfg::Q4) mma_commit(&wempty[w]);
+                if constexpr (Cfg::Q4) {
+                    mma_commit(&xempty[xs]);
+                    mma_commit(&wempty[w]);
+                } else {
+                    mma_commit(&rempty[s]);
+                }
                 if (last) {
                     mma_commit(&tfull[seg & 1]);
                     ++seg;
@@ -289,7 +329,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             if (!bounded_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, limit, p.status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                   acc * Cfg::NSUB * Cfg::MPAD;
+                                   acc * Cfg::ACC_COLS;
             // Partials are stored n-major, MS = M rounded up to 4 values per
             // column, so a thread writes and reads its columns with float4s.
             const int MS = (p.M + 3) & ~3;
@@ -308,7 +348,16 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     if (mc >= p.M) break;
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(taddr + j * Cfg::MPAD + mc, v);
+                    uint32_t vr[Cfg::R > 1 ? Cfg::R - 1 : 1][16];
+#pragma unroll
+                    for (int r = 1; r < Cfg::R; ++r)
+                        tmem_ld_32x32b_x16(taddr + (r * Cfg::NSUB + j) * Cfg::MPAD + mc, vr[r - 1]);
                     tmem_ld_wait();
+#pragma unroll
+                    for (int r = 1; r < Cfg::R; ++r)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(vr[r - 1][i]));
                     if (whole) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
