@@ -12,8 +12,11 @@
 //               columns 4 tn + j, 64 + 4 tn + j (j < 4): an 8 x 8 register
 //               tile.  Per 4 k-steps it reads 8 float4 of A (one per row,
 //               along k) and per k-step 2 float4 of B; each float4 pair feeds
-//               64 fp32 FMAs, issued as 32 paired FMAs (fma.rn.f32x2).  The swizzle makes the A reads of a warp (4 rows,
-//               same k chunk) hit 4 distinct bank groups.
+//               64 fp32 FMAs, issued as 32 paired FMAs (fma.rn.f32x2).  The
+//               fragments are double-buffered in registers, so the reads for
+//               the next k-step overlap the FMAs of this one.  The swizzle
+//               makes the A reads of a warp (4 rows, same k chunk) hit 4
+//               distinct bank groups.
 //   The accumulators go straight to global memory with float4 stores (a
 //   warp writes 4 rows x 128 contiguous bytes), clipped at the matrix edge.
 #include "ptx.cuh"
@@ -44,6 +47,21 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
     return v;
+}
+
+// The thread's 8 rows of A at 4-step group g of a slice: one float4 per row
+// (rows tm + 16 i; 128-byte rows, 16-byte unit g stored at unit g ^ (tm & 7)).
+__device__ __forceinline__ void load_a(uint32_t a_base, uint32_t xr, int g, float4 (&a)[8]) {
+    const uint32_t off = (static_cast<uint32_t>(g) ^ xr) << 4;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = lds128(a_base + i * 16 * 128 + off);
+}
+
+// The thread's 8 columns of one B row as 4 pairs: columns 4 tn .. 4 tn + 3
+// and 64 + 4 tn .. 64 + 4 tn + 3.
+__device__ __forceinline__ void load_b(uint32_t brow, uint64_t (&bp)[4]) {
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[0]), "=l"(bp[1]) : "r"(brow));
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[2]), "=l"(bp[3]) : "r"(brow + 256));
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -123,37 +141,50 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
     const uint32_t a_base0 = smem_u32(smA) + tm * 128;
     const uint32_t b_base0 = smem_u32(smB) + tn * 16;
+    // Register fragments are double-buffered: while the paired FMAs of k-step
+    // k issue, the A values of the next 4-step group and the B pairs of k + 1
+    // are already being read; at a slice's last k-step the first fragments of
+    // the next slice are read, so the math never waits on shared memory.
+    float4 a[2][8];          // [buffer][row i]: A[row][4 g .. 4 g + 3]
+    uint64_t bp[2][4];       // [buffer][pair j]: (B[k][2 j'], B[k][2 j' + 1])
+    if (num_kb > 0) {
+        if (!bounded_wait(&full[0], 0, abort_flag, p.timeout_ns, p.status)) return;
+        load_a(a_base0, xr, 0, a[0]);
+        load_b(b_base0, bp[0]);
+    }
     for (int kb = 0; kb < num_kb; ++kb) {
         const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!bounded_wait(&full[s], ph, abort_flag, p.timeout_ns, p.status)) break;
         const uint32_t a_base = a_base0 + s * A_STAGE;
         const uint32_t b_base = b_base0 + s * B_STAGE;
-#pragma unroll 2
-        for (int k4 = 0; k4 < BK / 4; ++k4) {
-            float4 a[8];
-            const uint32_t a_off = ((static_cast<uint32_t>(k4) ^ xr) << 4);
+        bool ok = true;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) a[i] = lds128(a_base + i * 16 * 128 + a_off);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t brow = b_base + (k4 * 4 + kk) * (BN * 4);
-                uint64_t bp[4];        // (B[k][2j], B[k][2j+1]) for the thread's 8 columns
-                asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[0]), "=l"(bp[1]) : "r"(brow));
-                asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(bp[2]), "=l"(bp[3]) : "r"(brow + 256));
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
-                    uint64_t aa;
-                    asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(av));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2[i][j]) : "l"(aa), "l"(bp[j]));
+        for (int k = 0; k < BK; ++k) {
+            if (k + 1 < BK) {
+                if (((k + 1) & 3) == 0) load_a(a_base, xr, (k + 1) >> 2, a[((k + 1) >> 2) & 1]);
+                load_b(b_base + (k + 1) * (BN * 4), bp[(k + 1) & 1]);
+            } else if (kb + 1 < num_kb) {
+                const int s2 = (kb + 1) % STAGES;
+                ok = bounded_wait(&full[s2], ((kb + 1) / STAGES) & 1, abort_flag, p.timeout_ns, p.status);
+                if (ok) {
+                    load_a(a_base0 + s2 * A_STAGE, xr, 0, a[0]);
+                    load_b(b_base0 + s2 * B_STAGE, bp[0]);
                 }
+            }
+            const float4 (&ak)[8] = a[(k >> 2) & 1];
+            const uint64_t (&bk)[4] = bp[k & 1];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float av = (k & 3) == 0 ? ak[i].x : (k & 3) == 1 ? ak[i].y : (k & 3) == 2 ? ak[i].z : ak[i].w;
+                uint64_t aa;
+                asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(av));
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2[i][j]) : "l"(aa), "l"(bk[j]));
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        if (!ok) break;
     }
     if (*abort_flag) return;
     float acc[8][8];
