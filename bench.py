@@ -380,6 +380,23 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(group, x, device):
+    """Largest value of x over all ranks (x itself when there is one rank)."""
+    if group is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    group.all_reduce(t, op=group.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step, steps, world, elapsed_max_s):
+    """Whole-job throughput: every rank processes the same units per step
+    (independent problems, weak scaling); the job takes as long as its
+    slowest rank."""
+    return units_per_rank_step * steps * world / elapsed_max_s
+
+
 def dist_setup(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -453,12 +470,6 @@ def main():
         if group is not None:
             group.barrier()
 
-    def max_over_ranks(x):
-        if group is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        group.all_reduce(t, op=group.ReduceOp.MAX)
-        return float(t.item())
 
     # ---------------------------------------------------------- headline
     case = Case(args.workload, dev, peaks)
@@ -486,12 +497,12 @@ def main():
         torch.cuda.synchronize()
         barrier()
     clocks = clk.summary()
-    elapsed = max_over_ranks(t_start.elapsed_time(t_end) * 1e-3)
+    elapsed = max_over_ranks(group, t_start.elapsed_time(t_end) * 1e-3, dev)
     launch_s = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_s, ev_e)])) * 1e-3
     st = tg.last_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} in timed region")
-    value = case.flops * K * ws / elapsed / 1e12      # whole-job TFLOP/s
+    value = job_rate(case.flops, K, ws, elapsed) / 1e12      # whole-job TFLOP/s
 
     # -------------------------------------------------------------- e2e
     pairs, host_out = case.host_pinned()
@@ -516,8 +527,8 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3)
-    e2e_val = case.flops * n_e2e * ws / e2e_s / 1e12
+    e2e_s = max_over_ranks(group, e0.elapsed_time(e1) * 1e-3, dev)
+    e2e_val = job_rate(case.flops, n_e2e, ws, e2e_s) / 1e12
 
     # -------------------------------------------------------- breakdown
     breakdown = []
@@ -557,6 +568,10 @@ def main():
         kind, M, N, Kd, seed, relu, dist_name = WORKLOADS[args.workload]
         traffic = traffic_record(args.workload)
         achieved = case.achieved(launch_s)
+        # the same peak measured as a seconds-long loop under the power cap
+        sustained = None
+        if case.unit == "TFLOP/s" and case.bound == "tensor" and "bf16_tflops_sustained" in peaks:
+            sustained = round(case.peak * peaks["bf16_tflops_sustained"] / peaks["bf16_tflops"], 1)
         line = {
             "metric": metric_name(), "value": round(value, 3), "unit": "TFLOP/s",
             "n_gpus": ws, "steps": K, "warmup": args.warmup,
@@ -570,6 +585,8 @@ def main():
                          "peak": case.peak, "unit": case.unit,
                          "frac": round(achieved / case.peak, 4),
                          "traffic": traffic, "peak_source": f"{peak_src} (burst)",
+                         "peak_sustained": sustained,
+                         "frac_of_sustained": (round(achieved / sustained, 4) if sustained else None),
                          "algorithmic_per_launch": case.flops if case.unit == "TFLOP/s"
                          else case.alg_bytes},
             "cpu_baseline": cpu,
