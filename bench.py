@@ -202,31 +202,80 @@ class Case:
 # ------------------------------------------------------------------ timing
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while running."""
+    """Samples the GPU's SM clock, power and clock-event reasons while the
+    timed region runs.  Read-only NVML queries from a background thread every
+    20 ms; the GPU is found by the CUDA device's PCI address, so the sampled
+    GPU is the one the bench runs on whatever the visible-device mapping.
+    Falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.02
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.stop = False
+
+    def _bus_id(self):
+        import torch
+        prop = torch.cuda.get_device_properties(self.gpu)
+        return f"{prop.pci_domain_id:08X}:{prop.pci_bus_id:02X}:{prop.pci_device_id:02X}.0"
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(self._bus_id())
+
+    def _poll(self, nv, h):
+        bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append(["0", str(sm), str(mx), str(pw), hex(r)] +
+                                 ["Active" if r & b else "Not Active" for b in bits])
+            except Exception:                        # stop sampling, keep what we have
+                return
+            time.sleep(self.PERIOD_S)
 
     def __enter__(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.rows and time.time() - t0 < 2.0:
+                time.sleep(0.005)
+            return self
+        except Exception:
+            self.thread = None
         import tempfile
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                ["nvidia-smi", "-i", self._bus_id(), f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except OSError:
+            t0 = time.time()                 # wait for the first sample
+            while os.path.getsize(self.path) == 0 and time.time() - t0 < 5.0:
+                time.sleep(0.05)
+        except Exception:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -235,15 +284,14 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.remove(self.path)
+        rows = list(self.rows)
+        if self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.remove(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
 
