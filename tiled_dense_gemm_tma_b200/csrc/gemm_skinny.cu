@@ -110,7 +110,7 @@ int run(const GemmArgs& a) {
     }
     const CUtensorMapDataType xt = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!tensor_map_2d(&tX, a.A, xt, 2, a.K, a.M, a.lda * 2, Cfg::BK, MPAD, SWZ_128))
+    if (!tensor_map_2d(&tX, a.A, xt, 2, a.K, a.M, a.lda * 2, 64, MPAD, SWZ_128))
         return kCudaError;
 
     auto kern = skinny_kernel<Cfg>;

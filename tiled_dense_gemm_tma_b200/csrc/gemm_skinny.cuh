@@ -8,7 +8,7 @@
 //
 //   D[n][m] = sum_k W[k][n] * X[m][k]        (C = D^T, X = A)
 //
-// * The weight tile (128 columns n x 64 rows k) is the MMA's 128-row operand,
+// * The weight tile (128 columns n x BK rows k) is the MMA's 128-row operand,
 //   N-major in shared memory; the activations (MPAD >= M rows, zero-padded
 //   by the copy engine) are the MMA's N operand, K-major.  D lives in TMEM as
 //   128 lanes (n) x MPAD columns (m).
@@ -37,15 +37,19 @@ struct SkCfg {
     static constexpr WKind W = W_;
     static constexpr int MPAD = MPAD_;                  // MMA N: 16, 32, 64 or 128
     static constexpr int TN = 128;                      // weight columns per MMA (MMA M)
-    static constexpr int BK = 64;                       // k rows per slice
     static constexpr bool Q4 = W_ == WKind::INT4;
+    // k rows per unit: 16-bit weights come in 128-row boxes (taller TMA
+    // copies stream faster), 4-bit weights in 64-row slices
+    static constexpr int BK = Q4 ? 64 : 128;
+    static constexpr int KSL = BK / 64;                 // 64-wide activation k-slices per unit
     // 4-bit units span two 128-column sub-tiles so packed rows arrive as
     // 128-byte runs (narrower rows stream markedly slower from HBM)
     static constexpr int NSUB = Q4 ? 2 : 1;
     static constexpr int GN = NSUB * TN;                // weight columns per unit
     static constexpr int W_CHUNK = BK * 128;            // 64 columns x BK rows, bytes
     static constexpr int W_BYTES = NSUB * 2 * W_CHUNK;  // fp16 weight tile of one unit
-    static constexpr int X_BYTES = MPAD * 128;          // MPAD rows x 64 fp16
+    static constexpr int X_SLICE = MPAD * 128;          // MPAD rows x 64 fp16
+    static constexpr int X_BYTES = KSL * X_SLICE;
     static constexpr int Q_BYTES = Q4 ? BK * GN / 2 : 0;   // 8 KB packed
     static constexpr int S_BYTES = Q4 ? GN * 2 : 0;        // 512 B scales
     // Ring of TMA-filled slots.  16-bit weights: [W | X], released by the MMA.
@@ -54,13 +58,18 @@ struct SkCfg {
     // travel in a ring of their own, released by the MMA.
     static constexpr int RAW_SLOT_USED = Q4 ? (Q_BYTES + S_BYTES) : (X_BYTES + W_BYTES);
     static constexpr int RAW_SLOT = (RAW_SLOT_USED + 1023) / 1024 * 1024;   // swizzle alignment
-    static constexpr int W_STAGES = Q4 ? 4 : 0;
+    // the fp16 tiles only bridge converters and MMA (on-chip latency): two
+    // suffice, which leaves the shared memory to packed weights in flight
+    static constexpr int W_STAGES = Q4 ? 2 : 0;
     static constexpr int X_STAGES = !Q4 ? 0 : (X_BYTES * 8 <= 32 * 1024 ? 8 : (32 * 1024) / X_BYTES);
     static constexpr int BUDGET = 212 * 1024 - W_STAGES * W_BYTES - X_STAGES * X_BYTES;
     static constexpr int RAW_STAGES_FIT = BUDGET / RAW_SLOT;
     static constexpr int RAW_STAGES = RAW_STAGES_FIT > 16 ? 16 : RAW_STAGES_FIT;
     static constexpr int EPI_WARPS = 4;
     static constexpr int CONV_WARPS = Q4 ? 8 : 0;
+    // rows per warp the reducer sums per round (registers allow more with the
+    // 6-warp 16-bit kernel than beside the 4-bit converters)
+    static constexpr int RED_ROWS = Q4 ? 2 : 8;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
     // Independent accumulator sets: k-step kk of a unit accumulates into set
     // kk % R, so consecutive small MMAs do not wait on each other's result;
@@ -108,6 +117,29 @@ __device__ __forceinline__ void store_out(void* C, long long ldc, int m, int n, 
         reinterpret_cast<__nv_bfloat16*>(C)[static_cast<long long>(m) * ldc + n] = __float2bfloat16_rn(v);
     } else {
         reinterpret_cast<__half*>(C)[static_cast<long long>(m) * ldc + n] = __float2half_rn(v);
+    }
+}
+
+// Four neighbouring outputs C[m][n .. n + 3] (n a multiple of 4): one 8-byte
+// store when all four are inside N (row pitches are multiples of 16 bytes).
+template <WKind W>
+__device__ __forceinline__ void store_out4(void* C, long long ldc, int m, int n, int N, const float (&o)[4]) {
+    if (n + 3 < N) {
+        uint2 pk;
+        if constexpr (W == WKind::BF16) {
+            __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]), b = __floats2bfloat162_rn(o[2], o[3]);
+            pk.x = *reinterpret_cast<uint32_t*>(&a);
+            pk.y = *reinterpret_cast<uint32_t*>(&b);
+        } else {
+            __half2 a = __floats2half2_rn(o[0], o[1]), b = __floats2half2_rn(o[2], o[3]);
+            pk.x = *reinterpret_cast<uint32_t*>(&a);
+            pk.y = *reinterpret_cast<uint32_t*>(&b);
+        }
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(C) + static_cast<long long>(m) * ldc + n) = pk;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (n + e < N) store_out<W>(C, ldc, m, n + e, o[e]);
     }
 }
 
@@ -221,7 +253,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     if (second)
                         tma_load_2d(slot_w(s) + Cfg::W_CHUNK, &tmW, &full[s], t * Cfg::TN + 64,
                                     kb * Cfg::BK);
-                    tma_load_2d(slot_x(s), &tmX, &full[s], kb * Cfg::BK, 0);
+#pragma unroll
+                    for (int ks = 0; ks < Cfg::KSL; ++ks)
+                        tma_load_2d(slot_x(s) + ks * Cfg::X_SLICE, &tmX, &full[s], kb * Cfg::BK + 64 * ks, 0);
                 }
                 armed |= 1u << s;
                 armed_par = (armed_par & ~(1u << s)) | (ph << s);
@@ -288,7 +322,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         // weights: N-major, 16 k rows of 128 B per MMA; activations: K-major
                         const uint64_t ad = sw128_desc(w_addr + j * 2 * Cfg::W_CHUNK + k * 16 * 128,
                                                        Cfg::W_CHUNK, 1024);
-                        const uint64_t bd = sw128_desc(x_addr + k * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(x_addr + (k >> 2) * Cfg::X_SLICE + (k & 3) * 32,
+                                                       16, 1024);
                         const int set = k % Cfg::R;
                         mma_f16(d_tmem + (set * Cfg::NSUB + j) * Cfg::MPAD, ad, bd, idesc,
                                 (first && k < Cfg::R) ? 0u : 1u);
@@ -330,9 +365,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    acc * Cfg::ACC_COLS;
-            // Partials are stored n-major, MS = M rounded up to 4 values per
-            // column, so a thread writes and reads its columns with float4s.
-            const int MS = (p.M + 3) & ~3;
+            // Partials are stored m-major (row m of GN fp32 per slot): the 32
+            // lanes of a warp hold 32 neighbouring columns, so each store and
+            // each reducer load covers whole 128-byte lines.
             const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::GN;
             float* slot = nullptr;
             if (!whole) {
@@ -367,13 +402,10 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                             if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
                         }
                     } else {
-                        float* col = slot + static_cast<long long>(nj) * MS;
+                        float* col = slot + nj;
 #pragma unroll
-                        for (int qd = 0; qd < 4; ++qd)
-                            if (mc + 4 * qd < MS)
-                                *reinterpret_cast<float4*>(col + mc + 4 * qd) =
-                                    make_float4(__uint_as_float(v[4 * qd]), __uint_as_float(v[4 * qd + 1]),
-                                                __uint_as_float(v[4 * qd + 2]), __uint_as_float(v[4 * qd + 3]));
+                        for (int i = 0; i < 16; ++i)
+                            if (mc + i < p.M) col[(mc + i) * Cfg::GN] = __uint_as_float(v[i]);
                     }
                 }
             }
@@ -401,50 +433,61 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             const int nseg = *last_flag;
             ++nsync;
             if (nseg) {
-                // Sum the tile's partials in segment order (deterministic) with
-                // up to 4 segments x 4 float4 loads in flight per thread.
+                // Sum the tile's partials in segment order (deterministic).
+                // Warp q takes rows m = q, q + 4, ...; each lane 4 neighbouring
+                // columns per 128-column chunk, so a load is 512 contiguous
+                // bytes; RR rows x up to 4 segments are in flight per round.
                 __threadfence();
-                const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::GN;
-                for (int j = 0; j < Cfg::NSUB; ++j) {
-                const int nj = j * Cfg::TN + n_loc;
-                const int n = t * Cfg::GN + nj;
-                const float* base = p.ws + static_cast<long long>(t) * p.J * sstride +
-                                    static_cast<long long>(nj) * MS;
-                for (int mb = 0; mb < MS; mb += 16) {
-                    float4 accv[4];
+                constexpr int CH = Cfg::GN / 128;             // 128-column chunks
+                constexpr int RR = Cfg::RED_ROWS;
+                const float* base = p.ws + static_cast<long long>(t) * p.J * sstride;
+                for (int m0 = q; m0 < p.M; m0 += 4 * RR) {
+                    float4 accv[RR][CH];
 #pragma unroll
-                    for (int qd = 0; qd < 4; ++qd) accv[qd] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int r = 0; r < RR; ++r)
+#pragma unroll
+                        for (int h = 0; h < CH; ++h) accv[r][h] = make_float4(0.f, 0.f, 0.f, 0.f);
                     for (int jj = 0; jj < nseg; jj += 4) {
-                        float4 vv[4][4];
+                        float4 vv[4][RR][CH];
 #pragma unroll
-                        for (int r = 0; r < 4; ++r)
+                        for (int g = 0; g < 4; ++g)
 #pragma unroll
-                            for (int qd = 0; qd < 4; ++qd)
-                                vv[r][qd] = (jj + r < nseg && mb + 4 * qd < MS)
-                                    ? __ldcg(reinterpret_cast<const float4*>(base + (jj + r) * sstride + mb + 4 * qd))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int r = 0; r < RR; ++r)
 #pragma unroll
-                        for (int r = 0; r < 4; ++r)
+                                for (int h = 0; h < CH; ++h) {
+                                    const int m = m0 + 4 * r;
+                                    vv[g][r][h] = (jj + g < nseg && m < p.M)
+                                        ? __ldcg(reinterpret_cast<const float4*>(
+                                              base + (jj + g) * sstride + static_cast<long long>(m) * Cfg::GN +
+                                              h * 128 + 4 * lane))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                                }
 #pragma unroll
-                            for (int qd = 0; qd < 4; ++qd) {
-                                accv[qd].x += vv[r][qd].x;
-                                accv[qd].y += vv[r][qd].y;
-                                accv[qd].z += vv[r][qd].z;
-                                accv[qd].w += vv[r][qd].w;
-                            }
+                        for (int g = 0; g < 4; ++g)
+#pragma unroll
+                            for (int r = 0; r < RR; ++r)
+#pragma unroll
+                                for (int h = 0; h < CH; ++h) {
+                                    accv[r][h].x += vv[g][r][h].x;
+                                    accv[r][h].y += vv[g][r][h].y;
+                                    accv[r][h].z += vv[g][r][h].z;
+                                    accv[r][h].w += vv[g][r][h].w;
+                                }
                     }
-                    if (n < p.N) {
 #pragma unroll
-                        for (int qd = 0; qd < 4; ++qd) {
-                            const float o[4] = {accv[qd].x, accv[qd].y, accv[qd].z, accv[qd].w};
+                    for (int r = 0; r < RR; ++r) {
+                        const int m = m0 + 4 * r;
+                        if (m >= p.M) break;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int m = mb + 4 * qd + e;
-                                if (m < p.M) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(o[e], 0.f) : o[e]);
-                            }
+                        for (int h = 0; h < CH; ++h) {
+                            const int n = t * Cfg::GN + h * 128 + 4 * lane;
+                            float o[4] = {accv[r][h].x, accv[r][h].y, accv[r][h].z, accv[r][h].w};
+                            if (p.relu)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) o[e] = fmaxf(o[e], 0.f);
+                            store_out4<Cfg::W>(p.C, p.ldc, m, n, p.N, o);
                         }
                     }
-                }
                 }
             }
         }
