@@ -2,6 +2,7 @@
 #include "launch.h"
 namespace tg {
 int launch_w4a16(const GemmArgs& a) {
+    if (a.M <= kGemvMaxM) return launch_gemv_w4a16(a);
     return a.M <= kSkinnyMaxM ? launch_skinny_w4a16(a) : launch_w4a16_large(a);
 }
 }

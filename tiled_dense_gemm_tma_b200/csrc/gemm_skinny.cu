@@ -29,8 +29,10 @@ struct Workspace {
 std::mutex g_ws_mu;
 std::map<std::pair<int, void*>, Workspace> g_ws;
 
-bool get_workspace(int dev, void* stream, long long tickets, long long partial_bytes,
-                   int** tk, float** part) {
+}  // namespace
+
+bool stream_workspace(int dev, void* stream, long long tickets, long long partial_bytes,
+                      int** tk, float** part) {
     std::lock_guard<std::mutex> lk(g_ws_mu);
     Workspace& w = g_ws[{dev, stream}];
     const long long tbytes = (tickets * 4 + 255) / 256 * 256;
@@ -63,6 +65,8 @@ bool get_workspace(int dev, void* stream, long long tickets, long long partial_b
     return true;
 }
 
+namespace {
+
 long long begin_of(long long c, long long U, long long G) { return c * U / G; }
 
 long long owner_of(long long u, long long U, long long G) {
@@ -90,7 +94,7 @@ int run(const GemmArgs& a) {
     }
     int* tickets = nullptr;
     float* ws = nullptr;
-    if (!get_workspace(dev, a.stream, T, T * J * MPAD * Cfg::GN * 4, &tickets, &ws))
+    if (!stream_workspace(dev, a.stream, T, T * J * MPAD * Cfg::GN * 4, &tickets, &ws))
         return kCudaError;
 
     CUtensorMap tW, tS, tX;

@@ -99,12 +99,12 @@ struct SkParams {
 };
 
 // First unit of CTA c's range.
-__device__ __forceinline__ int sk_begin(int c, int U, int G) {
+__host__ __device__ __forceinline__ int sk_begin(int c, int U, int G) {
     return static_cast<int>((static_cast<long long>(c) * U) / G);
 }
 
 // CTA whose range holds unit u.
-__device__ __forceinline__ int sk_owner(int u, int U, int G) {
+__host__ __device__ __forceinline__ int sk_owner(int u, int U, int G) {
     int c = static_cast<int>((static_cast<long long>(u) * G) / U);
     while (c + 1 < G && sk_begin(c + 1, U, G) <= u) ++c;
     while (c > 0 && sk_begin(c, U, G) > u) --c;

@@ -108,12 +108,14 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
 }  // namespace
 
 int launch_tc_bf16(const GemmArgs& a) {
+    if (a.M <= kGemvMaxM) return launch_gemv_bf16(a);
     if (a.M <= kSkinnyMaxM) return launch_skinny_bf16(a);
     const int r = run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
     if (r != kUnsupported) return r;
     return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
 }
 int launch_tc_f16(const GemmArgs& a) {
+    if (a.M <= kGemvMaxM) return launch_gemv_f16(a);
     if (a.M <= kSkinnyMaxM) return launch_skinny_f16(a);
     const int r = run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
     if (r != kUnsupported) return r;

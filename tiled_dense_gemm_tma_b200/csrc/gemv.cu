@@ -1,0 +1,460 @@
+// gemv.cu -- GEMM for one to four activation rows on the CUDA cores.
+//
+// With M <= 4 the product is a few dot products per weight column: the work
+// is streaming the K x N weight matrix once from HBM.  A tensor-core MMA
+// (at least 16 wide in M) would spend most of its operand traffic on padding
+// rows, and the 4-bit weights would have to be written back to shared memory
+// as fp16 for it.  Here the weights are multiplied where they land:
+//
+// * Stream-K split as in the weight-streaming tensor-core kernel: the units
+//   (GN columns x BK rows of weights) of all column groups are cut into one
+//   contiguous, equal range per SM; a maximal run of a range inside one
+//   column group is a segment.
+// * Warp 0 streams each unit by TMA into a ring of shared-memory slots: the
+//   weight tile (128-byte swizzled rows), for 4-bit weights the unit's fp16
+//   scale row, and the activations (MR rows x 64 values per slice).
+// * Sixteen CUDA-core warps (eight for four activation rows) read the slot:
+//   warp w takes a run of consecutive rows (vector reads fetch their
+//   activations); each lane its GN/32
+//   neighbouring columns of a row.  16-bit weights widen exactly to fp32 and
+//   multiply into fp32 accumulators.  Signed 4-bit weights decode exactly
+//   (nib_frac), and per unit a lane forms sum_k q[k][n] a[k] exactly-rounded
+//   in fp32, which the group scale s[g][n] multiplies once per unit (the
+//   dequantised weight W = q * s of the pages' dequantize GEMM, with the
+//   scale factored out of the unit's sum).
+// * At a segment's end the warps' sums are added in warp order through
+//   shared memory.  A segment that covers its whole column group writes C;
+//   otherwise the fp32 partial goes to a fixed workspace slot (row-major)
+//   and the CTA that takes the group's last ticket adds the slots in segment
+//   order -- deterministic -- applies ReLU, rounds and writes C.
+// Every wait is bounded (mbarriers, timeout -> device status 5).
+#include "gemm_skinny.cuh"   // WKind, SkParams, sk_begin / sk_owner, store_out4
+#include "host.cuh"
+#include "launch.h"
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace tg {
+
+namespace {
+
+template <WKind W_, int MR_>
+struct GvCfg {
+    static constexpr WKind W = W_;
+    static constexpr int MR = MR_;                      // activation rows: 1, 2 or 4
+    static constexpr bool Q4 = W_ == WKind::INT4;
+    static constexpr int GN = Q4 ? 256 : 128;           // columns per unit
+    static constexpr int BK = 128;                      // rows per unit (one scale group)
+    static constexpr int KSL = BK / 64;                 // 64-wide activation slices
+    static constexpr int CPL = GN / 32;                 // columns per lane
+    static constexpr int W_CHUNK = BK * 128;            // one 64-column box (16-bit)
+    static constexpr int W_BYTES = Q4 ? BK * GN / 2 : 2 * W_CHUNK;
+    static constexpr int S_BYTES = Q4 ? GN * 2 : 0;
+    static constexpr int X_SLICE = MR * 128;            // MR rows x 64 values
+    static constexpr int X_BYTES = KSL * X_SLICE;
+    static constexpr int SLOT = (W_BYTES + S_BYTES + X_BYTES + 1023) / 1024 * 1024;
+    // 16 math warps; 8 with four activation rows (their accumulators need
+    // more than the 96 registers a 544-thread CTA leaves per thread)
+    static constexpr int FMA_WARPS = MR_ == 4 ? 8 : 16;
+    static constexpr int FMA_THREADS = 32 * FMA_WARPS;
+    static constexpr int THREADS = 32 + FMA_THREADS;
+    static constexpr int RED_BYTES = FMA_WARPS * MR * GN * 4;
+    static constexpr int STAGES_FIT = (200 * 1024 - RED_BYTES) / SLOT;
+    static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
+    static constexpr int SMEM_BYTES = STAGES * SLOT + RED_BYTES + 512 + 1024;
+    static_assert(STAGES >= 3, "ring");
+};
+
+
+// Paired fp32 arithmetic (two independent IEEE operations per instruction,
+// each rounded as its scalar form).
+__device__ __forceinline__ uint64_t pk(float x, float y) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ void fma2(uint64_t& d, uint64_t x, uint64_t y) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(x), "l"(y));
+}
+
+// Exact decode of signed 4-bit weights to fp32 without a subtraction per
+// weight: with b = q + 8 in [0, 15] (the nibble with bit 3 flipped), the
+// float f = 1 + b / 16 is built by placing b under the exponent of 1.0
+// (bits 0x3F800000 | b << 19); f * a is exact for an fp16 activation a
+// (5 x 11 significant bits), and q = 16 f - 24, so
+//     sum_k q[k] a[k] = 16 sum_k f[k] a[k] - 24 sum_k a[k].
+// `t3` holds (b << 3) | 0x80 in each byte; byte i gives f.
+__device__ __forceinline__ float nib_frac(uint32_t t3, int i) {
+    return __uint_as_float(__byte_perm(t3, 0x3Fu, 0x4055u | (static_cast<uint32_t>(i) << 8)));
+}
+
+// Two activations (or 16-bit weights) packed in a word, widened to fp32.
+template <WKind T>
+__device__ __forceinline__ float2 widen2(uint32_t w) {
+    if constexpr (T == WKind::BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    else return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+gemv_kernel(const __grid_constant__ CUtensorMap tmW,
+            const __grid_constant__ CUtensorMap tmS,
+            const __grid_constant__ CUtensorMap tmX,
+            const SkParams p) {
+    constexpr int MR = Cfg::MR, GN = Cfg::GN, CPL = Cfg::CPL, BK = Cfg::BK;
+    constexpr WKind OUT = Cfg::Q4 ? WKind::F16 : Cfg::W;    // output / activation type
+    constexpr int ELEMS = MR * GN;                           // one segment's sums
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint8_t* ring = smem;                                            // STAGES x SLOT
+    float* red = reinterpret_cast<float*>(ring + Cfg::STAGES * Cfg::SLOT);  // [warp][m][column]
+    uint64_t* full = reinterpret_cast<uint64_t*>(red + Cfg::FMA_WARPS * ELEMS);
+    uint64_t* empty = full + Cfg::STAGES;
+    uint64_t* join = empty + Cfg::STAGES;                            // the FMA warps meet
+    uint64_t* flag = join + 1;                                       // ticket result published
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(flag + 1);
+    volatile int* last_flag = abort_flag + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = gridDim.x;
+    const int c = blockIdx.x;
+    const int u0 = sk_begin(c, p.U, G);
+    const int u1 = sk_begin(c + 1, p.U, G);
+    const int KB = p.KB;
+    const uint64_t limit = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], Cfg::FMA_WARPS);
+        }
+        mbar_init(join, Cfg::FMA_WARPS);
+        mbar_init(flag, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmW);
+            tma_prefetch_desc(&tmX);
+            if constexpr (Cfg::Q4) tma_prefetch_desc(&tmS);
+            uint32_t armed = 0, armed_par = 0;
+            bool ok = true;
+            int it = 0;
+            int t = u0 / KB, kb = u0 - (u0 / KB) * KB;      // unit u = t * KB + kb
+            for (int u = u0; u < u1; ++u, ++it, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0) {
+                const int s = it % Cfg::STAGES;
+                const uint32_t ph = (it / Cfg::STAGES) & 1;
+                if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                uint8_t* slot = ring + s * Cfg::SLOT;
+                uint8_t* xs = slot + Cfg::W_BYTES + Cfg::S_BYTES;
+                if constexpr (Cfg::Q4) {
+                    mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::S_BYTES + Cfg::X_BYTES);
+                    tma_load_2d(slot, &tmW, &full[s], t * (GN / 2), kb * BK);
+                    tma_load_2d(slot + Cfg::W_BYTES, &tmS, &full[s], t * GN, (kb * BK) / 128);
+                } else {
+                    // the second 64-column box is skipped when it starts past N
+                    // (its columns are never stored)
+                    const bool second = t * GN + 64 < p.N;
+                    mbar_arrive_expect_tx(&full[s], (second ? 2 : 1) * Cfg::W_CHUNK + Cfg::X_BYTES);
+                    tma_load_2d(slot, &tmW, &full[s], t * GN, kb * BK);
+                    if (second) tma_load_2d(slot + Cfg::W_CHUNK, &tmW, &full[s], t * GN + 64, kb * BK);
+                }
+                // the unit's activations: KSL slices of 64 values (X_BYTES in all)
+#pragma unroll
+                for (int ks = 0; ks < Cfg::KSL; ++ks)
+                    tma_load_2d(xs + ks * Cfg::X_SLICE, &tmX, &full[s], kb * BK + 64 * ks, 0);
+                armed |= 1u << s;
+                armed_par = (armed_par & ~(1u << s)) | (ph << s);
+            }
+            if (!ok) {
+                // let the copies in flight land before the CTA exits
+                for (int s = 0; s < Cfg::STAGES; ++s)
+                    if (armed & (1u << s)) {
+                        volatile int never = 0;
+                        bounded_wait(&full[s], (armed_par >> s) & 1, &never, limit, p.status);
+                    }
+            }
+        }
+        __syncwarp();
+    } else {
+        // -------------------------------------------------- CUDA-core warps
+        const int fw = warp - 1;                        // 0 .. FMA_WARPS - 1
+        const int ftid = threadIdx.x - 32;
+        uint32_t jphase = 0, fphase = 0;
+        // all FMA warps meet (bounded; false if the kernel is aborting)
+        auto join_all = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(join);
+            const bool ok = bounded_wait(join, jphase & 1, abort_flag, limit, p.status);
+            ++jphase;
+            return ok;
+        };
+        constexpr int RPW = BK / Cfg::FMA_WARPS;        // consecutive rows per warp and unit
+        const int r0 = fw * RPW;
+        float acc[MR][CPL];
+#pragma unroll
+        for (int m = 0; m < MR; ++m)
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) acc[m][q] = 0.f;
+        int it = 0;
+        int t = u0 / KB, kb = u0 - (u0 / KB) * KB;          // unit u = t * KB + kb
+        for (int u = u0; u < u1; ++u, ++it, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0) {
+            const int s = it % Cfg::STAGES;
+            const uint32_t ph = (it / Cfg::STAGES) & 1;
+            if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) break;
+            const uint8_t* slot = ring + s * Cfg::SLOT;
+            const uint8_t* xs = slot + Cfg::W_BYTES + Cfg::S_BYTES + (r0 >> 6) * Cfg::X_SLICE + (r0 & 63) * 2;
+            // activations of the warp's RPW rows: one vector read per m, kept
+            // packed (two values per word) and widened where used
+            uint32_t avw[MR][RPW / 2];
+#pragma unroll
+            for (int m = 0; m < MR; ++m)
+#pragma unroll
+                for (int h = 0; h < RPW / 8; ++h) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(xs + m * 128 + 16 * h);
+                    avw[m][4 * h] = v.x; avw[m][4 * h + 1] = v.y; avw[m][4 * h + 2] = v.z; avw[m][4 * h + 3] = v.w;
+                }
+            auto act = [&](int m, int i) -> float {
+                const float2 f = widen2<OUT>(avw[m][i >> 1]);
+                return (i & 1) ? f.y : f.x;
+            };
+            if constexpr (Cfg::Q4) {
+                uint64_t facc[MR][CPL / 2];                  // column pairs
+                float suma[MR];
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+                    suma[m] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < CPL / 2; ++q) facc[m][q] = 0ull;
+                }
+#pragma unroll
+                for (int i = 0; i < RPW; ++i) {
+                    const int r = r0 + i;
+                    // 4 bytes = columns 8 lane .. 8 lane + 7 of row r (16-byte
+                    // unit lane / 4, stored at unit (lane / 4) ^ (r % 8))
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                        slot + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
+                    const uint32_t tq = w ^ 0x88888888u;                          // b = q + 8
+                    const uint32_t te = ((tq << 3) & 0x78787878u) | 0x80808080u;  // columns 0, 2, 4, 6
+                    const uint32_t to = ((tq >> 1) & 0x78787878u) | 0x80808080u;  // columns 1, 3, 5, 7
+                    uint64_t a2[MR];                                               // (a, a)
+#pragma unroll
+                    for (int m = 0; m < MR; ++m) {
+                        const float am = act(m, i);
+                        a2[m] = pk(am, am);
+                        suma[m] += am;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        // columns (2 j, 2 j + 1) as one pair
+                        const uint64_t f2 = pk(nib_frac(te, j), nib_frac(to, j));
+#pragma unroll
+                        for (int m = 0; m < MR; ++m) fma2(facc[m][j], f2, a2[m]);
+                    }
+                }
+                // the unit's rows share one scale group: total += s * sum_k q a
+                const uint4 sv = *reinterpret_cast<const uint4*>(slot + Cfg::W_BYTES + lane * 16);
+                const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                float sc[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = widen2<WKind::F16>(sw[j]);
+                    sc[2 * j] = f.x;
+                    sc[2 * j + 1] = f.y;
+                }
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+                    const float nb = -24.f * suma[m];
+#pragma unroll
+                    for (int j = 0; j < CPL / 2; ++j) {
+                        const float2 f = upk(facc[m][j]);
+                        acc[m][2 * j] = fmaf(sc[2 * j], fmaf(16.f, f.x, nb), acc[m][2 * j]);
+                        acc[m][2 * j + 1] = fmaf(sc[2 * j + 1], fmaf(16.f, f.y, nb), acc[m][2 * j + 1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < RPW; ++i) {
+                    const int r = r0 + i;
+                    // 8 bytes = columns 4 lane .. 4 lane + 3: box lane / 16, 16-byte
+                    // unit (lane % 16) / 2 of the box row, stored at unit ^ (r % 8)
+                    const uint2 v = *reinterpret_cast<const uint2*>(
+                        slot + (lane >> 4) * Cfg::W_CHUNK + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) +
+                        (lane & 1) * 8);
+                    const float2 w0 = widen2<Cfg::W>(v.x), w1 = widen2<Cfg::W>(v.y);
+#pragma unroll
+                    for (int m = 0; m < MR; ++m) {
+                        const float am = act(m, i);
+                        acc[m][0] = fmaf(w0.x, am, acc[m][0]);
+                        acc[m][1] = fmaf(w0.y, am, acc[m][1]);
+                        acc[m][2] = fmaf(w1.x, am, acc[m][2]);
+                        acc[m][3] = fmaf(w1.y, am, acc[m][3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+
+            if (!(u == u1 - 1 || kb == KB - 1)) continue;
+            // ------------------------------------------------ segment end
+            const int sb = max(u0, t * KB);
+            const bool whole = sb == t * KB && u == t * KB + KB - 1;
+#pragma unroll
+            for (int m = 0; m < MR; ++m)
+#pragma unroll
+                for (int q = 0; q < CPL; q += 4) {
+                    *reinterpret_cast<float4*>(red + (fw * MR + m) * GN + lane * CPL + q) =
+                        make_float4(acc[m][q], acc[m][q + 1], acc[m][q + 2], acc[m][q + 3]);
+                    acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
+                }
+            if (!join_all()) break;
+            const int jseg = c - sk_owner(t * KB, p.U, G);
+            float* part = p.ws + (static_cast<long long>(t) * p.J + jseg) * ELEMS;
+            for (int e = ftid * 4; e < ELEMS; e += Cfg::FMA_THREADS * 4) {
+                float4 v = *reinterpret_cast<const float4*>(red + e);
+#pragma unroll
+                for (int w = 1; w < Cfg::FMA_WARPS; ++w) {
+                    const float4 x = *reinterpret_cast<const float4*>(red + w * ELEMS + e);
+                    v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                }
+                const int m = e / GN, col = e - (e / GN) * GN;
+                if (whole) {
+                    if (m < p.M) {
+                        float o[4] = {v.x, v.y, v.z, v.w};
+                        if (p.relu)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o[j] = fmaxf(o[j], 0.f);
+                        store_out4<OUT>(p.C, p.ldc, m, t * GN + col, p.N, o);
+                    }
+                } else {
+                    *reinterpret_cast<float4*>(part + e) = v;
+                }
+            }
+            __threadfence();
+            if (!join_all()) break;            // partials published, red free again
+            if (whole) continue;
+            if (ftid == 0) {
+                const int first = sk_owner(t * KB, p.U, G);
+                const int nseg = sk_owner(t * KB + KB - 1, p.U, G) - first + 1;
+                const int old = atomicAdd(&p.tickets[t], 1);
+                const int is_last = old == nseg - 1;
+                if (is_last) atomicExch(&p.tickets[t], 0);
+                *last_flag = is_last ? nseg : 0;
+                mbar_arrive(flag);
+            }
+            if (!bounded_wait(flag, fphase & 1, abort_flag, limit, p.status)) break;
+            ++fphase;
+            const int nseg = *last_flag;
+            if (!nseg) continue;
+            // the group's last contributor: add its partials in segment order
+            __threadfence();
+            const float* base = p.ws + static_cast<long long>(t) * p.J * ELEMS;
+            for (int e = ftid * 4; e < ELEMS; e += Cfg::FMA_THREADS * 4) {
+                const int m = e / GN, col = e - (e / GN) * GN;
+                if (m >= p.M) continue;
+                float4 v = __ldcg(reinterpret_cast<const float4*>(base + e));
+                for (int j = 1; j < nseg; ++j) {
+                    const float4 x = __ldcg(reinterpret_cast<const float4*>(base + static_cast<long long>(j) * ELEMS + e));
+                    v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                }
+                float o[4] = {v.x, v.y, v.z, v.w};
+                if (p.relu)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) o[j] = fmaxf(o[j], 0.f);
+                store_out4<OUT>(p.C, p.ldc, m, t * GN + col, p.N, o);
+            }
+        }
+    }
+    __syncthreads();
+}
+
+template <WKind W, int MR>
+int run_gemv(const GemmArgs& a) {
+    using Cfg = GvCfg<W, MR>;
+    int dev = 0;
+    const DeviceInfo* di = current_device(&dev);
+    if (!di) return kNoDevice;
+    const long long T = (a.N + Cfg::GN - 1) / Cfg::GN;
+    const long long KB = (a.K + Cfg::BK - 1) / Cfg::BK;
+    const long long U = T * KB;
+    if (U > 0x7fffffffll) return kUnsupported;
+    const long long G = U < di->num_sms ? U : di->num_sms;
+    long long J = 1;                              // most segments any column group has
+    for (long long t = 0; t < T; ++t) {
+        const long long n = sk_owner(static_cast<int>(t * KB + KB - 1), static_cast<int>(U), static_cast<int>(G)) -
+                            sk_owner(static_cast<int>(t * KB), static_cast<int>(U), static_cast<int>(G)) + 1;
+        if (n > J) J = n;
+    }
+    int* tickets = nullptr;
+    float* ws = nullptr;
+    if (!stream_workspace(dev, a.stream, T, T * J * MR * Cfg::GN * 4, &tickets, &ws)) return kCudaError;
+
+    const CUtensorMapDataType at = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap tW, tS, tX;
+    if constexpr (Cfg::Q4) {
+        if (!tensor_map_2d(&tW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
+                           Cfg::GN / 2, Cfg::BK, SWZ_128))
+            return kCudaError;
+        if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128, a.lds * 2,
+                           Cfg::GN, 1, SWZ_NONE))
+            return kCudaError;
+    } else {
+        if (!tensor_map_2d(&tW, a.B, at, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128)) return kCudaError;
+        tS = tW;                                   // unused
+    }
+    if (!tensor_map_2d(&tX, a.A, at, 2, a.K, a.M, a.lda * 2, 64, MR, SWZ_NONE)) return kCudaError;
+
+    auto kern = gemv_kernel<Cfg>;
+    const int slot = 40 + static_cast<int>(W) * 3 + (MR == 1 ? 0 : MR == 2 ? 1 : 2);
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return kCudaError;
+    SkParams p;
+    p.M = static_cast<int>(a.M);
+    p.N = static_cast<int>(a.N);
+    p.K = static_cast<int>(a.K);
+    p.relu = a.relu;
+    p.T = static_cast<int>(T);
+    p.KB = static_cast<int>(KB);
+    p.U = static_cast<int>(U);
+    p.J = static_cast<int>(J);
+    p.timeout_ns = wait_limit_ns();
+    p.status = device_status_ptr();
+    p.C = a.C;
+    p.ldc = a.ldc;
+    p.ws = ws;
+    p.tickets = tickets;
+    if (!p.status) return kCudaError;
+    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(
+        tW, tS, tX, p);
+    return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
+}
+
+template <WKind W>
+int dispatch_gemv(const GemmArgs& a) {
+    if (a.M <= 1) return run_gemv<W, 1>(a);
+    if (a.M <= 2) return run_gemv<W, 2>(a);
+    return run_gemv<W, 4>(a);
+}
+
+}  // namespace
+
+int launch_gemv_bf16(const GemmArgs& a) { return dispatch_gemv<WKind::BF16>(a); }
+int launch_gemv_f16(const GemmArgs& a) { return dispatch_gemv<WKind::F16>(a); }
+int launch_gemv_w4a16(const GemmArgs& a) { return dispatch_gemv<WKind::INT4>(a); }
+
+}  // namespace tg

@@ -29,8 +29,17 @@ int launch_w4a16_large(const GemmArgs& a);
 int launch_skinny_bf16(const GemmArgs& a);
 int launch_skinny_f16(const GemmArgs& a);
 int launch_skinny_w4a16(const GemmArgs& a);
+int launch_gemv_bf16(const GemmArgs& a);
+int launch_gemv_f16(const GemmArgs& a);
+int launch_gemv_w4a16(const GemmArgs& a);
 void mark_workspaces_dirty(int dev);
+// Per-(device, stream) scratch of the split-K paths: `tickets` ints (zero
+// between calls) and `partial_bytes` of fp32 partials.
+bool stream_workspace(int dev, void* stream, long long tickets, long long partial_bytes,
+                      int** tk, float** part);
 
+// Activation rows up to which the CUDA-core kernel is used.
+constexpr long long kGemvMaxM = 4;
 // Activation rows up to which the weight-streaming kernel is used.
 constexpr long long kSkinnyMaxM = 128;
 
