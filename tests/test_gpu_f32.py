@@ -85,3 +85,24 @@ def test_full_size_4096_sampled(tg, kind):
     else:
         assert rel_frob(got[rows], ref_r) <= 1e-5
         assert rel_frob(got[:, cols], ref_c) <= 1e-5
+
+
+@pytest.mark.parametrize("shape", [(200, 200, 3000), (129, 127, 1001), (64, 1000, 4096)])
+def test_split_k_shapes(tg, shape):
+    # fewer 128 x 128 tiles than SMs: K is split over several CTAs per tile
+    # (up to 8 ranges) and the partial tiles are added in range order
+    M, N, K = shape
+    A, B = synth.normal(M, N, K, seed=1)
+    for relu in (False, True):
+        got = _run(tg, A, B, relu)
+        assert rel_frob(got, oracle.gemm_f32(A, B, relu)) <= 1e-5
+
+
+def test_split_k_integer_bit_exact_and_repeatable(tg):
+    A, B = synth.integers(100, 300, 2048, seed=1)
+    got = _run(tg, A, B)
+    assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(A, B)))
+    A, B = synth.normal(1024, 1024, 1024, seed=1)
+    first = _run(tg, A, B)
+    for _ in range(3):
+        assert np.array_equal(_run(tg, A, B), first)

@@ -32,10 +32,13 @@ constexpr int A_STAGE = BM * BK * 4;     // 16 KB
 constexpr int B_STAGE = BK * BN * 4;     // 16 KB
 constexpr int COMPUTE_WARPS = 8;
 constexpr int THREADS = 32 * (COMPUTE_WARPS + 1);
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 128 + 1024;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 256 + 1024;
 
 struct FfmaParams {
     int M, N, K, ldc;
+    int splits;               // k ranges per output tile (blockIdx.z); 1 = no split
+    float* ws;                // splits > 1: [tile][split][BM][BN] fp32 partials
+    int* tickets;             // splits > 1: [tile], zero between calls
     int relu;
     unsigned long long timeout_ns;
     int* status;
@@ -75,11 +78,18 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint8_t* smB = smA + STAGES * A_STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(smB + STAGES * B_STAGE);
     uint64_t* empty = full + STAGES;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
+    uint64_t* join = empty + STAGES;                   // compute warps meet (split-K)
+    uint64_t* flag = join + 1;                         // ticket result published
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(flag + 1);
+    volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_kb = (p.K + BK - 1) / BK;
+    // this CTA's slices: [kb0, kb0 + nk) of the tile's k range
+    const int kb_all = (p.K + BK - 1) / BK;
+    const int kb_per = (kb_all + p.splits - 1) / p.splits;
+    const int kb0 = static_cast<int>(blockIdx.z) * kb_per;
+    const int num_kb = max(0, min(kb_all, kb0 + kb_per) - kb0);
     const int m0 = blockIdx.y * BM;
     const int n0 = blockIdx.x * BN;
 
@@ -88,7 +98,10 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], COMPUTE_WARPS);
         }
+        mbar_init(join, COMPUTE_WARPS);
+        mbar_init(flag, 1);
         *abort_flag = 0;
+        *last_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -111,8 +124,8 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
                 armed |= 1u << s;
                 armed_par = (armed_par & ~(1u << s)) | (ph << s);
-                tma_load_2d(smA + s * A_STAGE, &tmA, &full[s], kb * BK, m0);
-                tma_load_2d(smB + s * B_STAGE, &tmB, &full[s], n0, kb * BK);
+                tma_load_2d(smA + s * A_STAGE, &tmA, &full[s], (kb0 + kb) * BK, m0);
+                tma_load_2d(smB + s * B_STAGE, &tmB, &full[s], n0, (kb0 + kb) * BK);
             }
             if (!ok) {
                 for (int s = 0; s < STAGES; ++s)
@@ -195,26 +208,70 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[i][2 * j]), "=f"(acc[i][2 * j + 1]) : "l"(acc2[i][j]));
 
     // ---------------------------------------------------------- epilogue
+    // C[row][col .. col + 3] = epi(v), clipped at the matrix edge
+    auto store4 = [&](int row, int col, float4 q) {
+        if (row >= p.M) return;
+        float v[4] = {q.x, q.y, q.z, q.w};
+        if (p.relu)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int row = m0 + tm + 16 * i;
-        if (row >= p.M) continue;
+            for (int j = 0; j < 4; ++j) v[j] = fmaxf(v[j], 0.f);
         float* crow = p.C + static_cast<size_t>(row) * p.ldc;
+        if (col + 3 < p.N) {
+            *reinterpret_cast<float4*>(crow + col) = make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (col + j < p.N) crow[col + j] = v[j];
+        }
+    };
+    if (p.splits == 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                store4(m0 + tm + 16 * i, n0 + h * 64 + tn * 4,
+                       make_float4(acc[i][h * 4], acc[i][h * 4 + 1], acc[i][h * 4 + 2], acc[i][h * 4 + 3]));
+        return;
+    }
+    // Split K: publish this k range's partial tile and take the tile's
+    // ticket; the CTA of the last range adds the partials in range order
+    // (deterministic) and writes C.  The compute warps meet on mbarriers
+    // with bounded waits.
+    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+    float* part = p.ws + (static_cast<size_t>(tile) * p.splits + blockIdx.z) * (BM * BN);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            *reinterpret_cast<float4*>(part + (tm + 16 * i) * BN + h * 64 + tn * 4) =
+                make_float4(acc[i][h * 4], acc[i][h * 4 + 1], acc[i][h * 4 + 2], acc[i][h * 4 + 3]);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(join);
+    if (!bounded_wait(join, 0, abort_flag, p.timeout_ns, p.status)) return;
+    if (threadIdx.x == 0) {
+        const int old = atomicAdd(&p.tickets[tile], 1);
+        const int last = old == p.splits - 1;
+        if (last) atomicExch(&p.tickets[tile], 0);
+        *last_flag = last;
+        mbar_arrive(flag);
+    }
+    if (!bounded_wait(flag, 0, abort_flag, p.timeout_ns, p.status)) return;
+    if (!*last_flag) return;
+    __threadfence();
+    const float* base = p.ws + static_cast<size_t>(tile) * p.splits * (BM * BN);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int col = n0 + h * 64 + tn * 4;
-            float v[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = p.relu ? fmaxf(acc[i][h * 4 + j], 0.f) : acc[i][h * 4 + j];
-            if (col + 3 < p.N) {
-                *reinterpret_cast<float4*>(crow + col) = make_float4(v[0], v[1], v[2], v[3]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (col + j < p.N) crow[col + j] = v[j];
+            const int off = (tm + 16 * i) * BN + h * 64 + tn * 4;
+            float4 v = __ldcg(reinterpret_cast<const float4*>(base + off));
+            for (int z = 1; z < p.splits; ++z) {
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(base + static_cast<size_t>(z) * (BM * BN) + off));
+                v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
             }
+            store4(m0 + tm + 16 * i, n0 + h * 64 + tn * 4, v);
         }
-    }
 }
 
 }  // namespace
@@ -231,7 +288,28 @@ int launch_ffma_f32(const GemmArgs& a) {
         return kCudaError;
     if (set_smem_attr(reinterpret_cast<const void*>(ffma_gemm_kernel), SMEM_BYTES, 8) != cudaSuccess)
         return kCudaError;
+    const DeviceInfo* di = current_device(&dev);
+    const long long tiles_n = (a.N + BN - 1) / BN, tiles_m = (a.M + BM - 1) / BM;
+    const long long tiles = tiles_n * tiles_m;
+    const long long kb_all = (a.K + BK - 1) / BK;
+    // Fewer output tiles than SMs: split K so the grid fills the chip, with
+    // at least 8 slices (256 values of k) per range and at most 8 ranges.
+    long long splits = 1;
+    if (tiles < di->num_sms) {
+        splits = di->num_sms / tiles;
+        if (splits > kb_all / 8) splits = kb_all / 8;
+        if (splits > 8) splits = 8;
+        if (splits < 1) splits = 1;
+    }
+    int* tickets = nullptr;
+    float* ws = nullptr;
+    if (splits > 1 &&
+        !stream_workspace(dev, a.stream, tiles, tiles * splits * BM * BN * 4, &tickets, &ws))
+        return kCudaError;
     FfmaParams p;
+    p.splits = static_cast<int>(splits);
+    p.ws = ws;
+    p.tickets = tickets;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
@@ -242,7 +320,7 @@ int launch_ffma_f32(const GemmArgs& a) {
     p.C = static_cast<float*>(a.C);
     if (!p.status) return kCudaError;
     if (a.ldc > 0x7fffffff) return kUnsupported;
-    dim3 grid(static_cast<unsigned>((a.N + BN - 1) / BN), static_cast<unsigned>((a.M + BM - 1) / BM));
+    dim3 grid(static_cast<unsigned>(tiles_n), static_cast<unsigned>(tiles_m), static_cast<unsigned>(splits));
     if (grid.y > 65535) return kUnsupported;
     ffma_gemm_kernel<<<grid, THREADS, SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
