@@ -38,7 +38,10 @@ struct W4 {
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int GROUP_M = 16;
-    static constexpr int SMEM_DATA = RAW_STAGES * (A_BYTES + Q_BYTES + S_BYTES) +
+    // the scale ring is padded to 1 KB so the swizzled staging after it
+    // stays 1024-byte aligned
+    static constexpr int S_RING = (RAW_STAGES * S_BYTES + 1023) / 1024 * 1024;
+    static constexpr int SMEM_DATA = RAW_STAGES * (A_BYTES + Q_BYTES) + S_RING +
                                      B_STAGES * B_BYTES + EPI_WARPS * STG_BUF;
     static constexpr int SMEM_BYTES = SMEM_DATA + 256 + 1024;
 };
@@ -56,7 +59,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint8_t* smB = smA + W4::RAW_STAGES * W4::A_BYTES;
     uint8_t* smQ = smB + W4::B_STAGES * W4::B_BYTES;
     uint8_t* smS = smQ + W4::RAW_STAGES * W4::Q_BYTES;
-    uint8_t* smStg = smS + W4::RAW_STAGES * W4::S_BYTES;
+    uint8_t* smStg = smS + W4::S_RING;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smStg + W4::EPI_WARPS * W4::STG_BUF);
     uint64_t* full = bars;                               // [RAW_STAGES] TMA landed
     uint64_t* rempty = full + W4::RAW_STAGES;            // [RAW_STAGES] converters + MMA done
