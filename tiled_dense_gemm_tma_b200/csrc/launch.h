@@ -26,6 +26,7 @@ int launch_tc_tf32(const GemmArgs& a);
 int launch_ffma_f32(const GemmArgs& a);
 int launch_w4a16(const GemmArgs& a);
 int launch_w4a16_large(const GemmArgs& a);
+int launch_w4a16_pair(const GemmArgs& a);
 int launch_skinny_bf16(const GemmArgs& a);
 int launch_skinny_f16(const GemmArgs& a);
 int launch_skinny_w4a16(const GemmArgs& a);
