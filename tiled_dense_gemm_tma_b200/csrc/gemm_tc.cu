@@ -58,6 +58,7 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
 // kUnsupported (nothing launched) if the device refuses the cluster launch.
 template <class Cfg>
 int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
+    if (pair_kernels_disabled()) return kUnsupported;
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;

@@ -310,6 +310,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 // Returns kUnsupported (nothing launched) when the pair launch is refused,
 // so the caller can fall back to the one-CTA kernel.
 int launch_w4a16_pair(const GemmArgs& a) {
+    if (pair_kernels_disabled()) return kUnsupported;
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;

@@ -124,6 +124,14 @@ int inject_mode() {
     return v;
 }
 
+bool pair_kernels_disabled() {
+    static const bool v = [] {
+        const char* e = std::getenv("TG_NO_PAIR");
+        return e != nullptr && std::atoi(e) != 0;
+    }();
+    return v;
+}
+
 cudaError_t set_smem_attr(const void* func, int bytes, int slot) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -33,6 +33,10 @@ unsigned long long wait_limit_ns();
 
 // Debug fault-injection selector (TG_INJECT, default 0 = off).
 int inject_mode();
+// Debug: TG_NO_PAIR=1 makes every CTA-pair launch report "unsupported", so
+// the calls take the one-CTA kernels (the path used when a cluster launch is
+// refused).  Read once per process.
+bool pair_kernels_disabled();
 
 // Device address of the current device's status word (nullptr on error).
 int* device_status_ptr();
