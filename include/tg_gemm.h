@@ -34,7 +34,14 @@
  *   before any CUDA call; on any error nothing is launched and C is untouched.
  * - The library allocates no per-call memory.  It keeps, per device and for
  *   the life of the process, a small status word (see
- *   tg_last_device_status) and a cache of tensor-copy descriptors.
+ *   tg_last_device_status), a cache of tensor-copy descriptors, and one
+ *   split-K workspace per (device, stream): fp32 partials and tile tickets
+ *   of the kernels that split K across CTAs (M <= 128, and fp32 shapes with
+ *   fewer 128 x 128 tiles than SMs).  It is allocated on the first such call
+ *   on a stream (at least 8 MiB), grown when a larger call needs it (the
+ *   regrow frees the old one, which synchronises the device), and reused.
+ *   Calls on one stream share it; calls on different streams get their own.
+ *   tg_gemm_bf16_small_m_static avoids it.
  * - Thread safety: calls from several host threads are allowed.
  */
 #ifndef TG_GEMM_H
@@ -141,8 +148,9 @@ TG_API tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
  * latency-critical loop that must stay out of the driver's allocator).
  *
  * Same arguments, semantics and alignment rules as tg_gemm_bf16; M must be
- * <= 128 (else TG_ERR_UNSUPPORTED).  The split-K scratch of the small-M
- * kernel lives in a fixed device array of 16 MiB of fp32 partials plus 4096
+ * <= 128 (else TG_ERR_UNSUPPORTED).  It always runs the small-M tensor-core
+ * kernel (tg_gemm_bf16 takes a CUDA-core kernel for M <= 4).  The split-K
+ * scratch of that kernel lives in a fixed device array of 16 MiB of fp32 partials plus 4096
  * tile tickets that is part of the library image; shapes needing more return
  * TG_ERR_UNSUPPORTED.  Every call shares that array (tickets are cleared at
  * the start of each call): calls that overlap on the GPU, e.g. on two
