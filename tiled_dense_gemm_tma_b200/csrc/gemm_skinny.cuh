@@ -12,14 +12,16 @@
 //   N-major in shared memory; the activations (MPAD >= M rows, zero-padded
 //   by the copy engine) are the MMA's N operand, K-major.  D lives in TMEM as
 //   128 lanes (n) x MPAD columns (m).
-// * Stream-K: the (tile, k-slice) units of all T = ceil(N/128) tiles are cut
-//   into G (one per SM) contiguous, equal ranges.  A CTA accumulates each
-//   maximal run of its range inside one tile (a segment).  A segment that
-//   covers a whole tile is written to C directly; otherwise its fp32 partial
-//   goes to a workspace slot and the CTA that completes the tile's last
-//   segment (counted with an atomic ticket) sums the partials in segment
-//   order -- deterministic -- applies ReLU, rounds and writes C, and resets
-//   the ticket for the next call.
+// * Stream-K: the (column group, k-unit) units of all T = ceil(N/GN) column
+//   groups (GN = 128 columns, 256 for 4-bit weights; a unit is BK = 128
+//   rows of 16-bit or 64 rows of 4-bit weights) are cut into G (one per SM)
+//   contiguous, equal ranges.  A CTA accumulates each maximal run of its
+//   range inside one group (a segment).  A segment that covers a whole group
+//   is written to C directly; otherwise its fp32 partial goes to a workspace
+//   slot (row-major: row m of GN values) and the CTA that completes the
+//   group's last segment (counted with an atomic ticket) sums the partials
+//   in segment order -- deterministic -- applies ReLU, rounds and writes C,
+//   and resets the ticket for the next call.
 // * Weights arrive either as fp16/bf16 tiles by TMA, or as packed 4-bit
 //   weights + scales that converter warps expand (dequant.cuh).
 #pragma once
