@@ -113,6 +113,32 @@ TG_API tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
                        int epilogue, void *stream);
 
 /*
+ * tg_gemm_f16_ex, tg_gemm_bf16_ex -- C = epi(op(A) . op(B)) with optionally
+ * transposed operands, as the backward products of a linear layer need them
+ * (dA = dC . B^T, dB = A^T . dC; the autograd wrapper of the mhpq.cn article,
+ * section 3.4).  C is M x N row-major as in tg_gemm_f16.
+ *   trans_a = 0: A is M x K, row pitch lda >= K;  trans_a = 1: A is stored
+ *                K x M (op(A) = A^T), row pitch lda >= M.
+ *   trans_b = 0: B is K x N, row pitch ldb >= N;  trans_b = 1: B is stored
+ *                N x K (op(B) = B^T), row pitch ldb >= K.
+ * trans flags other than 0 / 1 -> TG_ERR_INVALID_ARG.  With both flags 0
+ * this is tg_gemm_f16 / tg_gemm_bf16.  A transposed call always runs the
+ * CTA-pair tensor-core kernel (no small-M variant), and returns
+ * TG_ERR_UNSUPPORTED if the device refuses its cluster launch.  Same
+ * alignment, status and ownership rules as tg_gemm_f16.
+ */
+TG_API tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K,
+                         const void *A, int64_t lda, int trans_a,
+                         const void *B, int64_t ldb, int trans_b,
+                         void *C, int64_t ldc,
+                         int epilogue, void *stream);
+TG_API tg_status tg_gemm_bf16_ex(int64_t M, int64_t N, int64_t K,
+                          const void *A, int64_t lda, int trans_a,
+                          const void *B, int64_t ldb, int trans_b,
+                          void *C, int64_t ldc,
+                          int epilogue, void *stream);
+
+/*
  * tg_gemm_w4a16 -- dequantize GEMM (the "Dequant GEMM" workload of the
  * blog.hotdry.top TileLang guide; the pages give no format, this library
  * defines it):  C = epi(A . W) with

@@ -91,3 +91,19 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(ImportError):
         binding.load_library()
+
+
+def _bf16_ex(lib, M, N, K, ta, tb, lda, ldb, ldc=None, A=P, B=P, C=P):
+    ldc = N if ldc is None else ldc
+    return lib.tg_gemm_bf16_ex(M, N, K, A, lda, ta, B, ldb, tb, C, ldc, 0, None)
+
+
+def test_argument_validation_transposed(lib):
+    # stored A is K x M when transposed: its pitch must cover M, not K
+    assert _bf16_ex(lib, 64, 32, 16, 1, 0, lda=56, ldb=32) == INVALID    # lda < M
+    assert _bf16_ex(lib, 64, 32, 16, 0, 1, lda=16, ldb=8) == INVALID     # ldb < K
+    assert _bf16_ex(lib, 64, 32, 16, 2, 0, lda=64, ldb=32) == INVALID    # flag not 0 / 1
+    assert _bf16_ex(lib, 64, 32, 16, 0, -1, lda=16, ldb=16) == INVALID
+    assert _bf16_ex(lib, 64, 32, 16, 1, 1, lda=64, ldb=20) == ALIGN      # 40-byte B pitch
+    assert _bf16_ex(lib, 0, 32, 16, 1, 1, lda=64, ldb=16) == OK          # empty output
+    assert lib.tg_gemm_f16_ex(64, 32, 16, P, 60, 1, P, 32, 0, P, 32, 0, None) == INVALID

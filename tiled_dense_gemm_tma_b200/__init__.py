@@ -2,7 +2,8 @@
 
 C = epi(A . B) with row-major A (M x K) and B (K x N), epi = identity or
 ReLU, in four precisions (fp32 FFMA or TF32, fp16, bf16, and 4-bit-weight
-dequantize GEMM).  All arithmetic runs in hand-written CUDA kernels behind a
+dequantize GEMM); 16-bit calls also take transposed operands, and
+``matmul`` is a differentiable 16-bit product built on them.  All arithmetic runs in hand-written CUDA kernels behind a
 C ABI (``include/tg_gemm.h``); this package is a thin ctypes binding that
 marshals torch tensors (device memory and streams only) into that ABI.
 
@@ -11,6 +12,6 @@ missing; there is no CPU or library fallback.
 """
 from .binding import (  # noqa: F401
     TgError, gemm_f32, gemm_f16, gemm_bf16, gemm_w4a16, gemm_bf16_small_m_static,
-    last_device_status,
+    matmul, last_device_status,
     lib_path, load_library, EPI_NONE, EPI_RELU, F32_FFMA, F32_TF32,
 )

@@ -20,7 +20,7 @@ STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
 
 # Every symbol include/tg_gemm.h declares.
 EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
-           "tg_gemm_bf16_small_m_static",
+           "tg_gemm_f16_ex", "tg_gemm_bf16_ex", "tg_gemm_bf16_small_m_static",
            "tg_status_string", "tg_last_device_status", "tg_num_sms")
 
 _lib = None
@@ -56,7 +56,10 @@ def load_library():
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, vp]
         lib.tg_gemm_w4a16.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
                                       vp, i64, ci, vp]
+        for name in ("tg_gemm_f16_ex", "tg_gemm_bf16_ex"):
+            getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, ci, vp, i64, ci, vp, i64, ci, vp]
         for name in ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
+                     "tg_gemm_f16_ex", "tg_gemm_bf16_ex",
                      "tg_gemm_bf16_small_m_static", "tg_last_device_status"):
             getattr(lib, name).restype = ci
         lib.tg_status_string.argtypes = [ci]
@@ -99,10 +102,10 @@ def empty_out(M, N, dtype, device):
     return torch.empty((M, ld), dtype=dtype, device=device)[:, :N]
 
 
-def _mk(A, B, C, dtype, out_dtype):
+def _mk(A, B, C, dtype, out_dtype, trans_a=False, trans_b=False):
     import torch
-    M, K = A.shape
-    K2, N = B.shape
+    M, K = A.shape[::-1] if trans_a else A.shape
+    K2, N = B.shape[::-1] if trans_b else B.shape
     if K != K2:
         raise ValueError(f"inner dimensions differ: {K} vs {K2}")
     for t, n in ((A, "A"), (B, "B")):
@@ -128,26 +131,72 @@ def gemm_f32(A, B, C=None, relu=False, mode=F32_FFMA, stream=None):
     return C
 
 
-def gemm_f16(A, B, C=None, relu=False, stream=None):
-    """C = epi(A @ B) for float16 CUDA tensors, fp32 accumulation."""
-    import torch
+def _gemm16(name, dtype, A, B, C, relu, stream, trans_a, trans_b):
     lib = load_library()
-    M, N, K, C = _mk(A, B, C, torch.float16, torch.float16)
-    _check(lib.tg_gemm_f16(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
-                           C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
-                           _stream_handle(stream)), "tg_gemm_f16")
+    M, N, K, C = _mk(A, B, C, dtype, dtype, trans_a, trans_b)
+    epi = EPI_RELU if relu else EPI_NONE
+    if trans_a or trans_b:
+        code = getattr(lib, name + "_ex")(M, N, K, A.data_ptr(), _ld(A, "A"), int(trans_a),
+                                         B.data_ptr(), _ld(B, "B"), int(trans_b),
+                                         C.data_ptr(), _ld(C, "C"), epi, _stream_handle(stream))
+        _check(code, name + "_ex")
+    else:
+        _check(getattr(lib, name)(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
+                                  C.data_ptr(), _ld(C, "C"), epi, _stream_handle(stream)), name)
     return C
 
 
-def gemm_bf16(A, B, C=None, relu=False, stream=None):
-    """C = epi(A @ B) for bfloat16 CUDA tensors, fp32 accumulation."""
+def gemm_f16(A, B, C=None, relu=False, stream=None, trans_a=False, trans_b=False):
+    """C = epi(op(A) @ op(B)) for float16 CUDA tensors, fp32 accumulation.
+
+    op(A) = A, or A.T when trans_a (A then holds the K x M matrix); op(B) =
+    B, or B.T when trans_b (B then holds N x K)."""
     import torch
-    lib = load_library()
-    M, N, K, C = _mk(A, B, C, torch.bfloat16, torch.bfloat16)
-    _check(lib.tg_gemm_bf16(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
-                            C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
-                            _stream_handle(stream)), "tg_gemm_bf16")
-    return C
+    return _gemm16("tg_gemm_f16", torch.float16, A, B, C, relu, stream, trans_a, trans_b)
+
+
+def gemm_bf16(A, B, C=None, relu=False, stream=None, trans_a=False, trans_b=False):
+    """C = epi(op(A) @ op(B)) for bfloat16 CUDA tensors, fp32 accumulation
+    (op as in gemm_f16)."""
+    import torch
+    return _gemm16("tg_gemm_bf16", torch.bfloat16, A, B, C, relu, stream, trans_a, trans_b)
+
+
+def _autograd_matmul():
+    import torch
+
+    class _Matmul(torch.autograd.Function):
+        """C = A @ B on this library's 16-bit kernels, with the backward
+        products dA = dC @ B^T and dB = A^T @ dC as transposed-operand calls
+        (no transposed copies are made)."""
+
+        @staticmethod
+        def forward(ctx, A, B):
+            ctx.save_for_backward(A, B)
+            fn = gemm_bf16 if A.dtype == torch.bfloat16 else gemm_f16
+            return fn(A, B)
+
+        @staticmethod
+        def backward(ctx, dC):
+            A, B = ctx.saved_tensors
+            fn = gemm_bf16 if A.dtype == torch.bfloat16 else gemm_f16
+            dC = dC.contiguous()
+            dA = fn(dC, B, trans_b=True) if ctx.needs_input_grad[0] else None
+            dB = fn(A, dC, trans_a=True) if ctx.needs_input_grad[1] else None
+            return dA, dB
+
+    return _Matmul
+
+
+_MATMUL = None
+
+
+def matmul(A, B):
+    """Differentiable C = A @ B for 2-D float16 / bfloat16 CUDA tensors."""
+    global _MATMUL
+    if _MATMUL is None:
+        _MATMUL = _autograd_matmul()
+    return _MATMUL.apply(A, B)
 
 
 def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None):

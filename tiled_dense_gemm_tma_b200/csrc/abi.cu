@@ -34,15 +34,18 @@ constexpr int64_t kMaxDim = (1ll << 31) - 1;      // kernel indices and TMA coor
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Shared checks for a plain GEMM with element size `eb` (bytes).
+// Shared checks for a GEMM with element size `eb` (bytes).  With trans_a
+// the stored A is K x M (rows of M), with trans_b the stored B is N x K.
 tg_status check_gemm(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
                      const void* B, int64_t ldb, const void* C, int64_t ldc,
-                     int epilogue, int eb) {
+                     int epilogue, int eb, int trans_a = 0, int trans_b = 0) {
     if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
     if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if ((trans_a != 0 && trans_a != 1) || (trans_b != 0 && trans_b != 1)) return TG_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return TG_OK;
     if (!C || ldc < N) return TG_ERR_INVALID_ARG;
-    if (K > 0 && (!A || !B || lda < K || ldb < N)) return TG_ERR_INVALID_ARG;
+    if (K > 0 && (!A || !B || lda < (trans_a ? M : K) || ldb < (trans_b ? K : N)))
+        return TG_ERR_INVALID_ARG;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
     if (!aligned16(C) || (ldc * eb) % 16 != 0) return TG_ERR_ALIGNMENT;
     if (K > 0 && (!aligned16(A) || !aligned16(B) || (lda * eb) % 16 != 0 || (ldb * eb) % 16 != 0))
@@ -99,6 +102,26 @@ tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K, const void* A, int64_t ld
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
     return static_cast<tg_status>(
         tg::launch_tc_f16(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream)));
+}
+
+tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int trans_a,
+                         const void* B, int64_t ldb, int trans_b, void* C, int64_t ldc,
+                         int epilogue, void* stream) {
+    tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2, trans_a, trans_b);
+    if (s != TG_OK || M == 0 || N == 0) return s;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    return static_cast<tg_status>(tg::launch_tc_trans(
+        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), 0, trans_a, trans_b));
+}
+
+tg_status tg_gemm_bf16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int trans_a,
+                          const void* B, int64_t ldb, int trans_b, void* C, int64_t ldc,
+                          int epilogue, void* stream) {
+    tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2, trans_a, trans_b);
+    if (s != TG_OK || M == 0 || N == 0) return s;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    return static_cast<tg_status>(tg::launch_tc_trans(
+        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), 1, trans_a, trans_b));
 }
 
 tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,

@@ -126,7 +126,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     if (!encode_map(&tW, B, N, K, ldb * 2, 64, Cfg::BK)) return TG_ERR_CUDA;
     if (!encode_map(&tX, A, K, M, lda * 2, 64, MPAD)) return TG_ERR_CUDA;
     auto kern = skinny_kernel<Cfg>;
-    const int slot = 40 + (MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3);
+    const int slot = 50 + (MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3);
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
         return TG_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -13,6 +13,13 @@ using CfgF16 = TcCfg<2, 0, OutT::F16, 256, 4>;
 using CfgTF32 = TcCfg<4, 2, OutT::F32, 256, 4>;
 using Cfg2BF16 = Tc2Cfg<1, OutT::BF16, 6>;
 using Cfg2F16 = Tc2Cfg<0, OutT::F16, 6>;
+// transposed operands (A stored K x M and/or B stored N x K)
+template <int FMT, OutT OUT>
+using Cfg2T10 = Tc2Cfg<FMT, OUT, 6, 1, 1>;
+template <int FMT, OutT OUT>
+using Cfg2T01 = Tc2Cfg<FMT, OUT, 6, 0, 0>;
+template <int FMT, OutT OUT>
+using Cfg2T11 = Tc2Cfg<FMT, OUT, 6, 1, 0>;
 
 template <class Cfg>
 int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, int slot) {
@@ -63,9 +70,15 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
     CUtensorMap tA, tB, tC;
-    if (!tensor_map_2d(&tA, a.A, dt, 2, a.K, a.M, a.lda * 2, Cfg::BK, Cfg::BM, SWZ_128))
+    // A: row-major M x K -> K-major boxes of BK x BM rows; stored transposed
+    // (K x M) -> M-major boxes of 64 rows of A x BK.
+    if (Cfg::A_MN ? !tensor_map_2d(&tA, a.A, dt, 2, a.M, a.K, a.lda * 2, 64, Cfg::BK, SWZ_128)
+                  : !tensor_map_2d(&tA, a.A, dt, 2, a.K, a.M, a.lda * 2, Cfg::BK, Cfg::BM, SWZ_128))
         return kCudaError;
-    if (!tensor_map_2d(&tB, a.B, dt, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128))
+    // B: row-major K x N -> N-major boxes of 64 columns x BK; stored
+    // transposed (N x K) -> K-major boxes of BK x HN columns.
+    if (Cfg::B_MN ? !tensor_map_2d(&tB, a.B, dt, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128)
+                  : !tensor_map_2d(&tB, a.B, dt, 2, a.K, a.N, a.ldb * 2, Cfg::BK, Cfg::HN, SWZ_128))
         return kCudaError;
     if (!tensor_map_2d(&tC, a.C, dt, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
         return kCudaError;
@@ -122,6 +135,20 @@ int launch_tc_f16(const GemmArgs& a) {
     if (r != kUnsupported) return r;
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
 }
+// 16-bit GEMM with optionally transposed operands: always the CTA-pair
+// kernel (no small-M or one-CTA variant); a refused cluster launch reports
+// kUnsupported.
+int launch_tc_trans(const GemmArgs& a, int bf16, int trans_a, int trans_b) {
+    if (!trans_a && !trans_b) return bf16 ? launch_tc_bf16(a) : launch_tc_f16(a);
+    const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (bf16) {
+        if (trans_a && trans_b) return run_pair<Cfg2T11<1, OutT::BF16>>(a, dt, 11);
+        return trans_a ? run_pair<Cfg2T10<1, OutT::BF16>>(a, dt, 12) : run_pair<Cfg2T01<1, OutT::BF16>>(a, dt, 13);
+    }
+    if (trans_a && trans_b) return run_pair<Cfg2T11<0, OutT::F16>>(a, dt, 14);
+    return trans_a ? run_pair<Cfg2T10<0, OutT::F16>>(a, dt, 15) : run_pair<Cfg2T01<0, OutT::F16>>(a, dt, 5);
+}
+
 int launch_tc_tf32(const GemmArgs& a) {
     return run<CfgTF32>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2);
 }

@@ -24,10 +24,16 @@
 
 namespace tg {
 
-template <int FMT_, OutT OUT_, int STAGES_>
+// A_MN_ = 1: A is stored transposed (K x M row-major), so its tiles arrive
+// M-major (64-row boxes along M) and the MMA reads A MN-major.  B_MN_ = 0: B
+// is stored transposed (N x K row-major) and is read K-major.  The default
+// (0, 1) is the row-major A (M x K) and B (K x N) of the plain GEMM.
+template <int FMT_, OutT OUT_, int STAGES_, int A_MN_ = 0, int B_MN_ = 1>
 struct Tc2Cfg {
     static constexpr int FMT = FMT_;
     static constexpr OutT OUT = OUT_;
+    static constexpr int A_MN = A_MN_;
+    static constexpr int B_MN = B_MN_;
     static constexpr int OUT_BYTES = 2;
     static constexpr int BM = 128;                      // rows per CTA
     static constexpr int PM = 256;                      // rows per pair tile
@@ -37,6 +43,7 @@ struct Tc2Cfg {
     static constexpr int MMA_K = 16;
     static constexpr int STAGES = STAGES_;
     static constexpr int A_STAGE = BM * 128;            // 16 KB
+    static constexpr int A_CHUNK = BK * 128;            // 8 KB: 64 rows of A x 64 k (M-major A)
     static constexpr int B_CHUNK = BK * 128;            // 8 KB: 64 columns x 64 rows
     static constexpr int B_STAGE = (HN / 64) * B_CHUNK; // 16 KB
     static constexpr int STG_BUF = 32 * 128;
@@ -115,9 +122,12 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const int n0 = tn * Cfg::BN + rank * Cfg::HN;
                 // boxes entirely past the matrix edge are not loaded: they only
                 // feed output rows / columns that are never stored
-                const bool a_live = m0 < p.M;
+                // 64-wide chunks (A rows or B columns) that start inside the matrix
+                const int a_live = m0 >= p.M ? 0 : (m0 + 64 < p.M ? 2 : 1);
                 const int b_live = n0 >= p.N ? 0 : (n0 + 64 < p.N ? 2 : 1);
-                const uint32_t bytes = (a_live ? Cfg::A_STAGE : 0) + b_live * Cfg::B_CHUNK;
+                const uint32_t a_bytes = Cfg::A_MN ? a_live * Cfg::A_CHUNK : (a_live ? Cfg::A_STAGE : 0);
+                const uint32_t b_bytes = Cfg::B_MN ? b_live * Cfg::B_CHUNK : (b_live ? Cfg::B_STAGE : 0);
+                const uint32_t bytes = a_bytes + b_bytes;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
@@ -127,11 +137,20 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     mbar_arrive_expect_tx_cluster(fbar, bytes);
                     armed |= 1u << s;
                     armed_par = (armed_par & ~(1u << s)) | (ph << s);
-                    if (a_live)
+                    if constexpr (Cfg::A_MN) {
+                        for (int j = 0; j < a_live; ++j)      // stored K x M: boxes of 64 rows of A
+                            tma_load_2d_pair(smA + s * Cfg::A_STAGE + j * Cfg::A_CHUNK, &tmA, fbar,
+                                             m0 + 64 * j, kb * Cfg::BK);
+                    } else if (a_live) {
                         tma_load_2d_pair(smA + s * Cfg::A_STAGE, &tmA, fbar, kb * Cfg::BK, m0);
-                    for (int j = 0; j < b_live; ++j)
-                        tma_load_2d_pair(smB + s * Cfg::B_STAGE + j * Cfg::B_CHUNK, &tmB, fbar,
-                                         n0 + 64 * j, kb * Cfg::BK);
+                    }
+                    if constexpr (Cfg::B_MN) {
+                        for (int j = 0; j < b_live; ++j)
+                            tma_load_2d_pair(smB + s * Cfg::B_STAGE + j * Cfg::B_CHUNK, &tmB, fbar,
+                                             n0 + 64 * j, kb * Cfg::BK);
+                    } else if (b_live) {                      // stored N x K: one box of 128 columns
+                        tma_load_2d_pair(smB + s * Cfg::B_STAGE, &tmB, fbar, kb * Cfg::BK, n0);
+                    }
                 }
             }
             if (!ok) {
@@ -153,7 +172,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // ------------------------------------------ MMA issuer (leader only)
         if (rank == 0 && elect_one()) {
-            constexpr uint32_t idesc = make_idesc(Cfg::FMT, Cfg::PM, Cfg::BN, 0, 1);
+            constexpr uint32_t idesc = make_idesc(Cfg::FMT, Cfg::PM, Cfg::BN, Cfg::A_MN, Cfg::B_MN);
             uint32_t it = 0, tl = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs, ++tl) {
@@ -171,8 +190,14 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t b_addr = smem_u32(smB + s * Cfg::B_STAGE);
 #pragma unroll
                     for (int k = 0; k < Cfg::BK / Cfg::MMA_K; ++k) {
-                        const uint64_t ad = sw128_desc(a_addr + k * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, 1024);
+                        // K-major: 16 k = 32 bytes along a 128-byte row; MN-major: 16 k
+                        // rows of 128 bytes, 64-wide chunks LBO apart
+                        const uint64_t ad = Cfg::A_MN
+                            ? sw128_desc(a_addr + k * Cfg::MMA_K * 128, Cfg::A_CHUNK, 1024)
+                            : sw128_desc(a_addr + k * 32, 16, 1024);
+                        const uint64_t bd = Cfg::B_MN
+                            ? sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, 1024)
+                            : sw128_desc(b_addr + k * 32, 16, 1024);
                         mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
                     }
                     const uint32_t e_loc = smem_u32(&empty[s]);

@@ -52,6 +52,15 @@ std::atomic<unsigned long long> g_attr_done[kMaxDevices];
 const DeviceInfo* current_device(int* dev_out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    // A host thread that has made no runtime call that binds a context (for
+    // example the autograd engine's worker thread) has no context current,
+    // and the driver-level tensor-map encoder then fails: make the device's
+    // primary context current on this thread once.
+    static thread_local int bound = -1;
+    if (bound != dev) {
+        if (cudaSetDevice(dev) != cudaSuccess) return nullptr;
+        bound = dev;
+    }
     std::call_once(g_dev_once[dev], [dev] {
         cudaDeviceProp prop;
         DeviceInfo info{0, 0};

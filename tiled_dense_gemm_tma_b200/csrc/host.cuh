@@ -42,6 +42,12 @@ bool pair_kernels_disabled();
 int* device_status_ptr();
 
 // Allow `func` to use `bytes` of dynamic shared memory (once per device).
+// `slot` (0..63) names the kernel in a per-device bitmask of done calls;
+// each kernel instantiation needs its own:
+//    0-4   gemm_tc.cu        one-CTA bf16/f16/tf32, CTA-pair bf16/f16
+//    5, 11-15 gemm_tc.cu     CTA-pair with transposed operands
+//    8     gemm_ffma.cu      9  gemm_w4a16.cu     10  gemm_w4a16_pair.cu
+//   16-27  gemm_skinny.cu    40-48  gemv.cu       50-53  gemm_skinny_static.cu
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 
 }  // namespace tg

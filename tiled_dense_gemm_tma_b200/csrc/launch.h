@@ -23,6 +23,7 @@ struct GemmArgs {
 int launch_tc_bf16(const GemmArgs& a);
 int launch_tc_f16(const GemmArgs& a);
 int launch_tc_tf32(const GemmArgs& a);
+int launch_tc_trans(const GemmArgs& a, int bf16, int trans_a, int trans_b);
 int launch_ffma_f32(const GemmArgs& a);
 int launch_w4a16(const GemmArgs& a);
 int launch_w4a16_large(const GemmArgs& a);
