@@ -62,8 +62,17 @@ WORKLOADS = {
     "w4a16_gemm_m16": ("w4a16", 16, 8192, 8192, 4, False, "w4a16"),
     "w4a16_gemm_m4096": ("w4a16", 4096, 8192, 8192, 4, False, "w4a16"),
 }
+# Transposed-operand variants: name -> (workload, A stored K x M, B stored N x K).
+# The same seeded matrices, stored transposed in HBM.
+TRANSPOSED = {
+    "bf16_gemm_8192_ta": ("bf16_gemm_8192", True, False),
+    "bf16_gemm_8192_tb": ("bf16_gemm_8192", False, True),
+    "bf16_gemm_8192_tatb": ("bf16_gemm_8192", True, True),
+    "bf16_gemm_16x8192x8192_tb": ("bf16_gemm_16x8192x8192", False, True),
+    "bf16_gemm_128x14336x4096_tb": ("bf16_gemm_128x14336x4096", False, True),
+}
 HEADLINE = "bf16_gemm_8192"
-BREAKDOWN = [w for w in WORKLOADS if w != HEADLINE]
+BREAKDOWN = [w for w in WORKLOADS if w != HEADLINE] + list(TRANSPOSED)
 
 
 def load_peaks():
@@ -132,9 +141,15 @@ class Case:
         import torch
         import tiled_dense_gemm_tma_b200 as tg
         self.name = name
-        kind, M, N, K, seed, relu, dist = WORKLOADS[name]
+        base, ta, tb = TRANSPOSED.get(name, (name, False, False))
+        kind, M, N, K, seed, relu, dist = WORKLOADS[base]
         self.kind, self.M, self.N, self.K, self.relu = kind, M, N, K, relu
-        host = make_inputs(name)
+        self.trans = (ta, tb)
+        host = make_inputs(base)
+        if ta:
+            host["A"] = np.ascontiguousarray(host["A"].T)
+        if tb:
+            host["B"] = np.ascontiguousarray(host["B"].T)
         self.flops = 2.0 * M * N * K
         if kind == "w4a16":
             self.A = _torch_of(host["A"], "f16", device)
@@ -159,9 +174,11 @@ class Case:
             self._host = host
             self._ik = ik
             if kind == "bf16":
-                self.run = lambda: tg.gemm_bf16(self.A, self.B, C=self.C, relu=relu)
+                self.run = lambda: tg.gemm_bf16(self.A, self.B, C=self.C, relu=relu,
+                                                trans_a=ta, trans_b=tb)
             elif kind == "f16":
-                self.run = lambda: tg.gemm_f16(self.A, self.B, C=self.C, relu=relu)
+                self.run = lambda: tg.gemm_f16(self.A, self.B, C=self.C, relu=relu,
+                                               trans_a=ta, trans_b=tb)
             else:
                 mode = tg.F32_TF32 if kind == "f32_tf32" else tg.F32_FFMA
                 self.run = lambda: tg.gemm_f32(self.A, self.B, C=self.C, relu=relu, mode=mode)
