@@ -1,0 +1,155 @@
+// Host checks of the work-distribution arithmetic the kernels share
+// (tile_sched.h): stream-K ranges, the weight-streaming launch plan, the
+// grouped tile raster and the fp32 split-K ranges.  Each entry point walks a
+// whole parameter grid, counts the properties it checked in *checked and
+// returns how many of them failed.  Built with g++ by test_sched_host.py.
+#include "tile_sched.h"
+
+#include <vector>
+
+using tg::sk_begin;
+using tg::sk_owner;
+
+extern "C" {
+
+// Ranges [sk_begin(c), sk_begin(c+1)) of U units over G CTAs: they tile
+// [0, U) in order, differ in size by at most one, are non-empty when G <= U,
+// and sk_owner(u) names the range that holds u.
+long long check_stream_k(int max_u, int max_g, long long* checked) {
+    long long bad = 0, n = 0;
+    for (int U = 1; U <= max_u; ++U) {
+        for (int G = 1; G <= max_g; ++G) {
+            const int lo = U / G, hi = (U + G - 1) / G;
+            ++n; bad += sk_begin(0, U, G) != 0;
+            ++n; bad += sk_begin(G, U, G) != U;
+            for (int c = 0; c < G; ++c) {
+                const int len = sk_begin(c + 1, U, G) - sk_begin(c, U, G);
+                ++n; bad += len < lo || len > hi;
+                if (G <= U) { ++n; bad += len == 0; }
+            }
+            for (int u = 0; u < U; ++u) {
+                const int c = sk_owner(u, U, G);
+                ++n;
+                bad += c < 0 || c >= G || sk_begin(c, U, G) > u || sk_begin(c + 1, U, G) <= u;
+            }
+        }
+    }
+    *checked = n;
+    return bad;
+}
+
+// The same near the int limit, where c * U overflows 32 bits.
+long long check_stream_k_large(long long* checked) {
+    long long bad = 0, n = 0;
+    const int Us[] = {2147483647, 2147483646, 1 << 30, 1000000007};
+    const int Gs[] = {1, 2, 147, 148, 296};
+    for (int U : Us) {
+        for (int G : Gs) {
+            long long prev = 0;
+            for (int c = 0; c < G; ++c) {
+                const long long b = sk_begin(c, U, G), e = sk_begin(c + 1, U, G);
+                ++n; bad += b != prev || e <= b;
+                ++n; bad += b != static_cast<long long>(c) * U / G;
+                ++n; bad += sk_owner(static_cast<int>(b), U, G) != c;
+                ++n; bad += sk_owner(static_cast<int>(e - 1), U, G) != c;
+                prev = e;
+            }
+            ++n; bad += prev != U;
+        }
+    }
+    *checked = n;
+    return bad;
+}
+
+// sk_plan against a brute-force walk: T and KB are ceilings, G = min(U,
+// num_sms), and J is the largest number of CTAs whose ranges touch one
+// column group's units, counted by walking every CTA's range unit by unit.
+long long check_sk_plan(long long* checked) {
+    long long bad = 0, n = 0;
+    const long long Ns[] = {1, 2, 127, 128, 129, 255, 256, 257, 1000, 4096, 8192, 14336};
+    const long long Ks[] = {1, 63, 64, 65, 128, 129, 1000, 4096, 8192};
+    const int gns[] = {128, 256};
+    const int bks[] = {64, 128};
+    const int smss[] = {1, 7, 148};
+    for (long long N : Ns) for (long long K : Ks) for (int gn : gns) for (int bk : bks)
+    for (int sms : smss) {
+        tg::SkPlan p;
+        ++n;
+        if (!tg::sk_plan(N, K, gn, bk, sms, &p)) { ++bad; continue; }
+        const long long T = (N + gn - 1) / gn, KB = (K + bk - 1) / bk, U = T * KB;
+        const long long G = U < sms ? U : sms;
+        ++n; bad += p.T != T || p.KB != KB || p.U != U || p.G != G;
+        std::vector<int> touching(T, 0), last(T, -1);
+        for (int c = 0; c < G; ++c) {
+            for (int u = sk_begin(c, int(U), int(G)); u < sk_begin(c + 1, int(U), int(G)); ++u) {
+                const long long t = u / KB;
+                if (last[t] != c) { last[t] = c; ++touching[t]; }
+            }
+        }
+        long long J = 1;
+        for (long long t = 0; t < T; ++t) J = touching[t] > J ? touching[t] : J;
+        ++n; bad += p.J != J;
+    }
+    // unit counts past the int range are refused
+    tg::SkPlan p;
+    ++n; bad += tg::sk_plan(1ll << 40, 1ll << 20, 128, 128, 148, &p);
+    *checked = n;
+    return bad;
+}
+
+// tile_coords maps [0, ntm*ntn) one-to-one onto the tile grid, keeps index t
+// in band t / (group_m * ntn), and inside a band steps down a tile column
+// before moving to the next column.
+long long check_tile_coords(int max_ntm, int max_ntn, long long* checked) {
+    long long bad = 0, n = 0;
+    const int groups[] = {1, 2, 3, 4, 8, 16};
+    for (int ntm = 1; ntm <= max_ntm; ++ntm) for (int ntn = 1; ntn <= max_ntn; ++ntn)
+    for (int gm : groups) {
+        std::vector<char> seen(static_cast<size_t>(ntm) * ntn, 0);
+        int ptm = -1, ptn = -1;
+        for (int t = 0; t < ntm * ntn; ++t) {
+            int tm, tn;
+            tg::tile_coords(t, ntm, ntn, gm, tm, tn);
+            ++n;
+            if (tm < 0 || tm >= ntm || tn < 0 || tn >= ntn) { ++bad; continue; }
+            char& s = seen[static_cast<size_t>(tm) * ntn + tn];
+            ++n; bad += s != 0;
+            s = 1;
+            const int band = t / (gm * ntn);
+            ++n; bad += tm / gm != band;
+            if (t > 0 && t % (gm * ntn) != 0) {
+                const bool down = tn == ptn && tm == ptm + 1;
+                const bool next_col = tn == ptn + 1 && tm == band * gm;
+                ++n; bad += !(down || next_col);
+            }
+            ptm = tm; ptn = tn;
+        }
+    }
+    *checked = n;
+    return bad;
+}
+
+// ffma_splits stays in [1, 8], is 1 when the tiles fill the SMs, never asks
+// for more CTAs than SMs or fewer than 8 k-slices per range on average, and
+// its ranges tile [0, kb_all) in order with none empty.
+long long check_ffma_splits(int max_tiles, int max_kb, int num_sms, long long* checked) {
+    long long bad = 0, n = 0;
+    for (int tiles = 1; tiles <= max_tiles; ++tiles) for (int kb = 1; kb <= max_kb; ++kb) {
+        const int s = tg::ffma_splits(tiles, kb, num_sms);
+        ++n; bad += s < 1 || s > 8;
+        if (tiles >= num_sms) { ++n; bad += s != 1; }
+        if (s > 1) { ++n; bad += static_cast<long long>(s) * tiles > num_sms || s > kb / 8; }
+        const int per = tg::ffma_kb_per(kb, s);
+        int next = 0;
+        for (int z = 0; z < s; ++z) {
+            const int b = z * per, len = tg::ffma_range_len(b, per, kb);
+            ++n; bad += b != next || len <= 0 || len > per;
+            next = b + len;
+        }
+        ++n; bad += next != kb;
+    }
+    *checked = n;
+    return bad;
+}
+
+}  // extern "C"

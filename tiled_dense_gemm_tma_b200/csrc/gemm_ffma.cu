@@ -20,6 +20,7 @@
 //   The accumulators go straight to global memory with float4 stores (a
 //   warp writes 4 rows x 128 contiguous bytes), clipped at the matrix edge.
 #include "ptx.cuh"
+#include "tile_sched.h"
 #include "host.cuh"
 #include "launch.h"
 
@@ -85,11 +86,11 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // this CTA's slices: [kb0, kb0 + nk) of the tile's k range
+    // this CTA's slices: [kb0, kb0 + num_kb) of the tile's k range
     const int kb_all = (p.K + BK - 1) / BK;
-    const int kb_per = (kb_all + p.splits - 1) / p.splits;
+    const int kb_per = ffma_kb_per(kb_all, p.splits);
     const int kb0 = static_cast<int>(blockIdx.z) * kb_per;
-    const int num_kb = max(0, min(kb_all, kb0 + kb_per) - kb0);
+    const int num_kb = ffma_range_len(kb0, kb_per, kb_all);
     const int m0 = blockIdx.y * BM;
     const int n0 = blockIdx.x * BN;
 
@@ -292,15 +293,8 @@ int launch_ffma_f32(const GemmArgs& a) {
     const long long tiles_n = (a.N + BN - 1) / BN, tiles_m = (a.M + BM - 1) / BM;
     const long long tiles = tiles_n * tiles_m;
     const long long kb_all = (a.K + BK - 1) / BK;
-    // Fewer output tiles than SMs: split K so the grid fills the chip, with
-    // at least 8 slices (256 values of k) per range and at most 8 ranges.
-    long long splits = 1;
-    if (tiles < di->num_sms) {
-        splits = di->num_sms / tiles;
-        if (splits > kb_all / 8) splits = kb_all / 8;
-        if (splits > 8) splits = 8;
-        if (splits < 1) splits = 1;
-    }
+    // Fewer output tiles than SMs: split K so the grid fills the chip.
+    const long long splits = ffma_splits(tiles, kb_all, di->num_sms);
     int* tickets = nullptr;
     float* ws = nullptr;
     if (splits > 1 &&

@@ -27,6 +27,7 @@
 #pragma once
 #include "ptx.cuh"
 #include "dequant.cuh"
+#include "tile_sched.h"     // sk_begin / sk_owner
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -96,22 +97,9 @@ struct SkParams {
     int* status;
     void* C;
     long long ldc;
-    float* ws;                // [T][J] slots of MPAD*GN fp32: column-major partials
+    float* ws;                // [T][J] slots of MPAD*GN fp32: row-major partials (row m: GN values)
     int* tickets;             // [T], zero between calls
 };
-
-// First unit of CTA c's range.
-__host__ __device__ __forceinline__ int sk_begin(int c, int U, int G) {
-    return static_cast<int>((static_cast<long long>(c) * U) / G);
-}
-
-// CTA whose range holds unit u.
-__host__ __device__ __forceinline__ int sk_owner(int u, int U, int G) {
-    int c = static_cast<int>((static_cast<long long>(u) * G) / U);
-    while (c + 1 < G && sk_begin(c + 1, U, G) <= u) ++c;
-    while (c > 0 && sk_begin(c, U, G) > u) --c;
-    return c;
-}
 
 template <WKind W>
 __device__ __forceinline__ void store_out(void* C, long long ldc, int m, int n, float v) {

@@ -65,15 +65,6 @@ bool static_scratch(int dev, float** part, int** tick) {
     return true;
 }
 
-long long sbegin(long long c, long long U, long long G) { return c * U / G; }
-
-long long sowner(long long u, long long U, long long G) {
-    long long c = u * G / U;
-    while (c + 1 < G && sbegin(c + 1, U, G) <= u) ++c;
-    while (c > 0 && sbegin(c, U, G) > u) --c;
-    return c;
-}
-
 // A tensor map encoded directly (no cache insertion, so no host allocation).
 typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -107,16 +98,9 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
                      const void* B, int64_t ldb, void* C, int64_t ldc, int relu,
                      void* stream, const DeviceInfo* di, int dev) {
     using Cfg = SkCfg<WKind::BF16, MPAD>;
-    const long long T = (N + Cfg::GN - 1) / Cfg::GN;
-    const long long KB = (K + Cfg::BK - 1) / Cfg::BK;
-    const long long U = T * KB;
-    if (U > 0x7fffffffll) return TG_ERR_UNSUPPORTED;
-    const long long G = U < di->num_sms ? U : di->num_sms;
-    long long J = 1;
-    for (long long t = 0; t < T; ++t) {
-        const long long n = sowner(t * KB + KB - 1, U, G) - sowner(t * KB, U, G) + 1;
-        if (n > J) J = n;
-    }
+    SkPlan pl;
+    if (!sk_plan(N, K, Cfg::GN, Cfg::BK, di->num_sms, &pl)) return TG_ERR_UNSUPPORTED;
+    const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
     if (T > kStaticTickets || T * J * MPAD * Cfg::GN > kStaticPartialFloats)
         return TG_ERR_UNSUPPORTED;                     // beyond the fixed scratch size
     float* part = nullptr;

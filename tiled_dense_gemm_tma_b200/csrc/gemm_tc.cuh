@@ -32,6 +32,7 @@
 // locality of the blog.hotdry.top guide).  The grid is one CTA per SM.
 #pragma once
 #include "ptx.cuh"
+#include "tile_sched.h"     // tile_coords
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -104,18 +105,6 @@ __device__ __forceinline__ void store_row_tail(uint8_t* dst, const uint4* packed
             }
         }
     }
-}
-
-// Map a linear tile index to (tile_m, tile_n), GROUP_M tile rows per band.
-__device__ __forceinline__ void tile_coords(int t, int ntm, int ntn, int group_m,
-                                            int& tm, int& tn) {
-    const int per_group = group_m * ntn;
-    const int g = t / per_group;
-    const int first_m = g * group_m;
-    const int gsz = min(ntm - first_m, group_m);
-    const int local = t - g * per_group;
-    tm = first_m + local % gsz;
-    tn = local / gsz;
 }
 
 // Source position, inside an 8-column group, of output column q when the

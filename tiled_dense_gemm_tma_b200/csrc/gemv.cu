@@ -388,17 +388,9 @@ int run_gemv(const GemmArgs& a) {
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
-    const long long T = (a.N + Cfg::GN - 1) / Cfg::GN;
-    const long long KB = (a.K + Cfg::BK - 1) / Cfg::BK;
-    const long long U = T * KB;
-    if (U > 0x7fffffffll) return kUnsupported;
-    const long long G = U < di->num_sms ? U : di->num_sms;
-    long long J = 1;                              // most segments any column group has
-    for (long long t = 0; t < T; ++t) {
-        const long long n = sk_owner(static_cast<int>(t * KB + KB - 1), static_cast<int>(U), static_cast<int>(G)) -
-                            sk_owner(static_cast<int>(t * KB), static_cast<int>(U), static_cast<int>(G)) + 1;
-        if (n > J) J = n;
-    }
+    SkPlan pl;
+    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK, di->num_sms, &pl)) return kUnsupported;
+    const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
     int* tickets = nullptr;
     float* ws = nullptr;
     if (!stream_workspace(dev, a.stream, T, T * J * MR * Cfg::GN * 4, &tickets, &ws)) return kCudaError;
