@@ -26,7 +26,9 @@
  * - stream is a cudaStream_t passed as void*; NULL means the legacy default
  *   stream.  Calls are asynchronous: they validate, enqueue and return.
  * - Sizes: M, N, K >= 0.  M == 0 or N == 0 -> TG_OK, nothing is launched.
- *   K == 0 -> C = epi(0) = 0 is written.
+ *   K == 0 -> C = epi(0) = 0 is written.  M, N, K above 2^31 - 1, or a row
+ *   pitch (ld * sizeof(element)) of 2^40 bytes or more -> TG_ERR_UNSUPPORTED
+ *   (the limits of the kernels' 32-bit indices and of a TMA stride).
  * - Alignment (the hardware tensor-copy engine, TMA, needs 16-byte aligned
  *   bases and row pitches): every base pointer 16-byte aligned and every
  *   ld * sizeof(element) a multiple of 16 bytes, else TG_ERR_ALIGNMENT.
@@ -42,7 +44,9 @@
  *   regrow frees the old one, which synchronises the device), and reused.
  *   Calls on one stream share it; calls on different streams get their own.
  *   tg_gemm_bf16_small_m_static avoids it.
- * - Thread safety: calls from several host threads are allowed.
+ * - Thread safety: calls from several host threads are allowed.  A thread
+ *   needs no earlier CUDA call: on its first call the library makes the
+ *   current device's primary context current on that thread.
  */
 #ifndef TG_GEMM_H
 #define TG_GEMM_H

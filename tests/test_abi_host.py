@@ -86,6 +86,25 @@ def test_argument_validation_w4a16(lib):
     assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 3, None) == INVALID
 
 
+def test_row_pitch_limits(lib):
+    """Row pitches of 2^40 bytes or more are refused before any product
+    ld * sizeof(element) is formed, so even pitches near 2^63 are reported
+    as TG_ERR_UNSUPPORTED rather than wrapping into a small value."""
+    huge = (1 << 62) + 8                       # * 2 or * 4 would overflow int64
+    at_limit = (1 << 39)                       # 2^40 bytes of bf16
+    assert _bf16(lib, 8, 8, 8, ldc=at_limit) == UNSUP
+    assert _bf16(lib, 8, 8, 8, lda=huge) == UNSUP
+    assert _bf16(lib, 8, 8, 8, ldb=huge) == UNSUP
+    assert _bf16(lib, 8, 8, 8, ldc=huge) == UNSUP
+    f = lib.tg_gemm_f32
+    assert f(8, 8, 8, P, 1 << 38, P, 8, P, 8, 0, 0, None) == UNSUP   # 2^40 bytes of fp32
+    w = lib.tg_gemm_w4a16
+    assert w(4, 32, 256, P, 256, P, 1 << 40, P, 32, 128, P, 32, 0, None) == UNSUP   # ldbq
+    assert w(4, 32, 256, P, 256, P, 16, P, huge, 128, P, 32, 0, None) == UNSUP      # lds
+    assert w(4, 32, 256, P, huge, P, 16, P, 32, 128, P, 32, 0, None) == UNSUP       # lda
+    assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, huge, 0, None) == UNSUP      # ldc
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_HERE", str(tmp_path))
     monkeypatch.setattr(binding, "_lib", None)

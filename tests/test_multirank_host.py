@@ -56,7 +56,7 @@ def test_two_gloo_ranks_agree_on_max_time(tmp_path):
     world = 2
     mp.start_processes(rank_main, args=(world, free_port(), str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
-    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    res = [json.loads((tmp_path / f"rank{r}.json").read_text()) for r in range(world)]
     for r in res:
         assert r["elapsed"] == 2.0                      # the slowest rank's time
         assert r["rate"] == 2e12 * 10 * world / 2.0     # all ranks' work / max time

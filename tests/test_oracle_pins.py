@@ -48,7 +48,8 @@ def _np_f16_decode(bits):
 
 def _np_bf16_decode(bits):
     u = np.asarray(bits, np.uint16).astype(np.uint32) << 16
-    return u.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):         # signalling-NaN patterns are expected here
+        return u.view(np.float32).astype(np.float64)
 
 
 def _exact(Ad, Bd):

@@ -9,21 +9,25 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace tg {
 
 // Per-device status word written by kernels whose bounded wait expired.
 __device__ int g_device_status = 0;
 
 int* device_status_ptr() {
-    static int* ptrs[64] = {};
+    static std::atomic<int*> ptrs[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
+    int* q = ptrs[dev].load(std::memory_order_acquire);
+    if (!q) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<int*>(p);
+        q = static_cast<int*>(p);
+        ptrs[dev].store(q, std::memory_order_release);   // every thread finds the same address
     }
-    return ptrs[dev];
+    return q;
 }
 
 }  // namespace tg
@@ -33,6 +37,10 @@ namespace {
 constexpr int64_t kMaxDim = (1ll << 31) - 1;      // kernel indices and TMA coords are int32
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A row pitch of ld elements of eb bytes that a tensor map can take: TMA
+// strides stay below 2^40 bytes.  Checked before any ld * eb product.
+bool pitch_ok(int64_t ld, int eb) { return ld < (1ll << 40) / eb; }
 
 // Shared checks for a GEMM with element size `eb` (bytes).  With trans_a
 // the stored A is K x M (rows of M), with trans_b the stored B is N x K.
@@ -47,12 +55,11 @@ tg_status check_gemm(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     if (K > 0 && (!A || !B || lda < (trans_a ? M : K) || ldb < (trans_b ? K : N)))
         return TG_ERR_INVALID_ARG;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!pitch_ok(ldc, eb) || (K > 0 && (!pitch_ok(lda, eb) || !pitch_ok(ldb, eb))))
+        return TG_ERR_UNSUPPORTED;
     if (!aligned16(C) || (ldc * eb) % 16 != 0) return TG_ERR_ALIGNMENT;
     if (K > 0 && (!aligned16(A) || !aligned16(B) || (lda * eb) % 16 != 0 || (ldb * eb) % 16 != 0))
         return TG_ERR_ALIGNMENT;
-    // TMA strides must stay below 2^40 bytes.
-    if (ldc * eb >= (1ll << 40) || lda * eb >= (1ll << 40) || ldb * eb >= (1ll << 40))
-        return TG_ERR_UNSUPPORTED;
     return TG_OK;
 }
 
@@ -145,6 +152,9 @@ tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K, const void* A, int64_t 
     if (K > 0 && (!A || !Bq || !scales || lda < K || ldbq < (N + 1) / 2 || lds < N))
         return TG_ERR_INVALID_ARG;
     if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!pitch_ok(ldc, 2) ||
+        (K > 0 && (!pitch_ok(lda, 2) || !pitch_ok(ldbq, 1) || !pitch_ok(lds, 2))))
+        return TG_ERR_UNSUPPORTED;
     if (!aligned16(C) || (ldc * 2) % 16 != 0) return TG_ERR_ALIGNMENT;
     if (K > 0 && (!aligned16(A) || !aligned16(Bq) || !aligned16(scales) || (lda * 2) % 16 != 0 ||
                   ldbq % 16 != 0 || (lds * 2) % 16 != 0))
