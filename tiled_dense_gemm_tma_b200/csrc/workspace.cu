@@ -7,14 +7,17 @@
 
 #include <map>
 #include <mutex>
-#include <utility>
+#include <thread>
+#include <tuple>
 
 namespace tg {
 
 namespace {
 
 // One workspace per (device, stream): calls on one stream run in order, so
-// they can share it; calls on different streams get their own.  Layout:
+// they can share it; calls on different streams get their own.  The handle
+// cudaStreamPerThread names a different stream on every host thread, so for
+// it the calling thread is part of the key.  Layout:
 // [tickets: ticket_cap ints, zeroed][partials: partial_cap bytes].  Tickets
 // return to zero at the end of every complete call; a call that timed out
 // can leave them dirty, so a device-status read that reports a timeout marks
@@ -26,15 +29,22 @@ struct Workspace {
     bool dirty = false;
 };
 
+using WsKey = std::tuple<int, void*, std::thread::id>;
+
 std::mutex g_ws_mu;
-std::map<std::pair<int, void*>, Workspace> g_ws;
+std::map<WsKey, Workspace> g_ws;
+
+WsKey ws_key(int dev, void* stream) {
+    const bool per_thread = stream == static_cast<void*>(cudaStreamPerThread);
+    return WsKey(dev, stream, per_thread ? std::this_thread::get_id() : std::thread::id());
+}
 
 }  // namespace
 
 bool stream_workspace(int dev, void* stream, long long tickets, long long partial_bytes,
                       int** tk, float** part) {
     std::lock_guard<std::mutex> lk(g_ws_mu);
-    Workspace& w = g_ws[{dev, stream}];
+    Workspace& w = g_ws[ws_key(dev, stream)];
     if (!w.base || w.ticket_cap < tickets || w.partial_cap < partial_bytes) {
         if (w.base) {
             cudaFree(w.base);     // synchronises the device: no kernel still uses it
@@ -66,7 +76,7 @@ bool stream_workspace(int dev, void* stream, long long tickets, long long partia
 void mark_workspaces_dirty(int dev) {
     std::lock_guard<std::mutex> lk(g_ws_mu);
     for (auto& kv : g_ws)
-        if (kv.first.first == dev) kv.second.dirty = true;
+        if (std::get<0>(kv.first) == dev) kv.second.dirty = true;
 }
 
 }  // namespace tg
