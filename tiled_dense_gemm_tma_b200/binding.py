@@ -4,6 +4,7 @@ Argument marshalling only: every step of the GEMM runs in the CUDA kernels
 of ``libtg_gemm.so``.  Torch is used for device memory and streams.  If the
 library is missing, the first call raises; there is no fallback.
 """
+import contextlib
 import ctypes
 import os
 import threading
@@ -80,6 +81,25 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _require_cuda(device, *named):
+    """Every tensor on `device`, a CUDA device: the kernels run on the device
+    that holds the operands and take raw device pointers."""
+    for t, n in named:
+        if not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+        if t.device != device:
+            raise ValueError(f"{n} is on {t.device}, the operands on {device}")
+
+
+def _device_ctx(t):
+    """Make t's device current for the call (the library launches on the
+    current device; the default stream is that device's current stream)."""
+    if not t.is_cuda:
+        return contextlib.nullcontext()
+    import torch
+    return torch.cuda.device(t.device)
+
+
 def _ld(t, name):
     """Row pitch (elements) of a row-major 2-D tensor view."""
     if t.dim() != 2:
@@ -103,7 +123,8 @@ def empty_out(M, N, dtype, device):
 
 
 def _mk(A, B, C, dtype, out_dtype, trans_a=False, trans_b=False):
-    import torch
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D")
     M, K = A.shape[::-1] if trans_a else A.shape
     K2, N = B.shape[::-1] if trans_b else B.shape
     if K != K2:
@@ -111,12 +132,12 @@ def _mk(A, B, C, dtype, out_dtype, trans_a=False, trans_b=False):
     for t, n in ((A, "A"), (B, "B")):
         if t.dtype != dtype:
             raise TypeError(f"{n} must be {dtype}")
-        if not t.is_cuda:
-            raise ValueError(f"{n} must be a CUDA tensor")
+    _require_cuda(A.device, (A, "A"), (B, "B"))
     if C is None:
         C = empty_out(M, N, out_dtype, A.device)
     elif C.shape != (M, N) or C.dtype != out_dtype:
         raise ValueError("C has the wrong shape or dtype")
+    _require_cuda(A.device, (C, "C"))
     return M, N, K, C
 
 
@@ -125,9 +146,11 @@ def gemm_f32(A, B, C=None, relu=False, mode=F32_FFMA, stream=None):
     import torch
     lib = load_library()
     M, N, K, C = _mk(A, B, C, torch.float32, torch.float32)
-    _check(lib.tg_gemm_f32(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
-                           C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
-                           mode, _stream_handle(stream)), "tg_gemm_f32")
+    with _device_ctx(A):
+        code = lib.tg_gemm_f32(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
+                               C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                               mode, _stream_handle(stream))
+    _check(code, "tg_gemm_f32")
     return C
 
 
@@ -135,14 +158,17 @@ def _gemm16(name, dtype, A, B, C, relu, stream, trans_a, trans_b):
     lib = load_library()
     M, N, K, C = _mk(A, B, C, dtype, dtype, trans_a, trans_b)
     epi = EPI_RELU if relu else EPI_NONE
-    if trans_a or trans_b:
-        code = getattr(lib, name + "_ex")(M, N, K, A.data_ptr(), _ld(A, "A"), int(trans_a),
-                                         B.data_ptr(), _ld(B, "B"), int(trans_b),
-                                         C.data_ptr(), _ld(C, "C"), epi, _stream_handle(stream))
-        _check(code, name + "_ex")
-    else:
-        _check(getattr(lib, name)(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(), _ld(B, "B"),
-                                  C.data_ptr(), _ld(C, "C"), epi, _stream_handle(stream)), name)
+    with _device_ctx(A):
+        if trans_a or trans_b:
+            name += "_ex"
+            code = getattr(lib, name)(M, N, K, A.data_ptr(), _ld(A, "A"), int(trans_a),
+                                      B.data_ptr(), _ld(B, "B"), int(trans_b),
+                                      C.data_ptr(), _ld(C, "C"), epi, _stream_handle(stream))
+        else:
+            code = getattr(lib, name)(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(),
+                                      _ld(B, "B"), C.data_ptr(), _ld(C, "C"), epi,
+                                      _stream_handle(stream))
+    _check(code, name)
     return C
 
 
@@ -162,27 +188,59 @@ def gemm_bf16(A, B, C=None, relu=False, stream=None, trans_a=False, trans_b=Fals
     return _gemm16("tg_gemm_bf16", torch.bfloat16, A, B, C, relu, stream, trans_a, trans_b)
 
 
+def _row_major(t):
+    return t.stride(1) == 1 or t.shape[1] <= 1
+
+
+def _stored(u):
+    """How the logical 2-D matrix u reaches the kernels: (storage, transposed)
+    with u == storage or u == storage.T and the storage row-major.  A
+    transposed view (e.g. W.T of a row-major W) needs no copy.  Where both
+    readings hold, the one with a 16-byte row pitch wins, the plain one
+    first; a view that is neither is copied to a contiguous tensor."""
+    cands = []
+    if _row_major(u) and u.stride(0) >= u.shape[1]:
+        cands.append((u, False))
+    v = u.t()
+    if _row_major(v) and v.stride(0) >= v.shape[1]:
+        cands.append((v, True))
+    for st, tr in cands:
+        if (st.stride(0) * st.element_size()) % 16 == 0:
+            return st, tr
+    if cands:
+        return cands[0]
+    return u.contiguous(), False
+
+
 def _autograd_matmul():
     import torch
 
     class _Matmul(torch.autograd.Function):
         """C = A @ B on this library's 16-bit kernels, with the backward
-        products dA = dC @ B^T and dB = A^T @ dC as transposed-operand calls
-        (no transposed copies are made)."""
+        products dA = dC @ B^T and dB = A^T @ dC.  Every operand, the
+        gradient included, is passed as it is stored: a transposed view
+        becomes a transposed-operand call, not a copy."""
 
         @staticmethod
         def forward(ctx, A, B):
             ctx.save_for_backward(A, B)
             fn = gemm_bf16 if A.dtype == torch.bfloat16 else gemm_f16
-            return fn(A, B)
+            a, ta = _stored(A)
+            b, tb = _stored(B)
+            return fn(a, b, trans_a=ta, trans_b=tb)
 
         @staticmethod
         def backward(ctx, dC):
             A, B = ctx.saved_tensors
             fn = gemm_bf16 if A.dtype == torch.bfloat16 else gemm_f16
-            dC = dC.contiguous()
-            dA = fn(dC, B, trans_b=True) if ctx.needs_input_grad[0] else None
-            dB = fn(A, dC, trans_a=True) if ctx.needs_input_grad[1] else None
+            g, tg = _stored(dC)
+            dA = dB = None
+            if ctx.needs_input_grad[0]:
+                x, tx = _stored(B.t())
+                dA = fn(g, x, trans_a=tg, trans_b=tx)
+            if ctx.needs_input_grad[1]:
+                y, ty = _stored(A.t())
+                dB = fn(y, g, trans_a=ty, trans_b=tg)
             return dA, dB
 
     return _Matmul
@@ -192,7 +250,11 @@ _MATMUL = None
 
 
 def matmul(A, B):
-    """Differentiable C = A @ B for 2-D float16 / bfloat16 CUDA tensors."""
+    """Differentiable C = A @ B for 2-D float16 / bfloat16 CUDA tensors.
+
+    A and B may be row-major or transposed views of row-major storage (such
+    as W.T for a linear layer's out x in weight W); both reach the kernels
+    without a copy."""
     global _MATMUL
     if _MATMUL is None:
         _MATMUL = _autograd_matmul()
@@ -209,15 +271,23 @@ def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None
     lib = load_library()
     if A.dtype != torch.float16 or scales.dtype != torch.float16 or Bq.dtype != torch.uint8:
         raise TypeError("A and scales must be float16, Bq uint8")
+    if A.dim() != 2 or Bq.dim() != 2 or scales.dim() != 2:
+        raise ValueError("A, Bq and scales must be 2-D")
     M, K = A.shape
     if Bq.shape[0] != K:
         raise ValueError("Bq must have K rows")
+    _require_cuda(A.device, (A, "A"), (Bq, "Bq"), (scales, "scales"))
     if C is None:
         C = empty_out(M, N, torch.float16, A.device)
-    _check(lib.tg_gemm_w4a16(M, N, K, A.data_ptr(), _ld(A, "A"), Bq.data_ptr(), _ld(Bq, "Bq"),
-                             scales.data_ptr(), _ld(scales, "scales"), group_size,
-                             C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
-                             _stream_handle(stream)), "tg_gemm_w4a16")
+    elif C.shape != (M, N) or C.dtype != torch.float16:
+        raise ValueError("C has the wrong shape or dtype")
+    _require_cuda(A.device, (C, "C"))
+    with _device_ctx(A):
+        code = lib.tg_gemm_w4a16(M, N, K, A.data_ptr(), _ld(A, "A"), Bq.data_ptr(),
+                                 _ld(Bq, "Bq"), scales.data_ptr(), _ld(scales, "scales"),
+                                 group_size, C.data_ptr(), _ld(C, "C"),
+                                 EPI_RELU if relu else EPI_NONE, _stream_handle(stream))
+    _check(code, "tg_gemm_w4a16")
     return C
 
 
@@ -228,10 +298,12 @@ def gemm_bf16_small_m_static(A, B, C=None, relu=False, stream=None):
     import torch
     lib = load_library()
     M, N, K, C = _mk(A, B, C, torch.bfloat16, torch.bfloat16)
-    _check(lib.tg_gemm_bf16_small_m_static(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(),
-                                           _ld(B, "B"), C.data_ptr(), _ld(C, "C"),
-                                           EPI_RELU if relu else EPI_NONE, _stream_handle(stream)),
-           "tg_gemm_bf16_small_m_static")
+    with _device_ctx(A):
+        code = lib.tg_gemm_bf16_small_m_static(M, N, K, A.data_ptr(), _ld(A, "A"), B.data_ptr(),
+                                               _ld(B, "B"), C.data_ptr(), _ld(C, "C"),
+                                               EPI_RELU if relu else EPI_NONE,
+                                               _stream_handle(stream))
+    _check(code, "tg_gemm_bf16_small_m_static")
     return C
 
 
