@@ -105,6 +105,26 @@ def test_row_pitch_limits(lib):
     assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, huge, 0, None) == UNSUP      # ldc
 
 
+def test_valid_calls_without_a_device_report_no_device(lib):
+    """On a machine with no GPU a well-formed call gets past validation and
+    must report TG_ERR_NO_DEVICE (no CPU fallback, no crash).  The fake
+    pointers must never reach a kernel, so this runs only where the library
+    itself sees no device."""
+    if lib.tg_num_sms() >= 0:
+        pytest.skip("a CUDA device is present")
+    NODEV = 6
+    assert _bf16(lib, 64, 64, 64) == NODEV
+    assert lib.tg_gemm_f16(64, 64, 64, P, 64, P, 64, P, 64, 0, None) == NODEV
+    for mode in (0, 1):
+        assert lib.tg_gemm_f32(64, 64, 64, P, 64, P, 64, P, 64, 0, mode, None) == NODEV
+    assert lib.tg_gemm_w4a16(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 0, None) == NODEV
+    assert lib.tg_gemm_bf16_ex(64, 64, 64, P, 64, 1, P, 64, 1, P, 64, 0, None) == NODEV
+    assert lib.tg_gemm_f16_ex(64, 64, 64, P, 64, 0, P, 64, 1, P, 64, 0, None) == NODEV
+    assert lib.tg_gemm_bf16_small_m_static(16, 64, 64, P, 64, P, 64, P, 64, 0, None) == NODEV
+    # K == 0 writes C = 0 with a device memset: also no device here
+    assert _bf16(lib, 8, 8, 0) == NODEV
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_HERE", str(tmp_path))
     monkeypatch.setattr(binding, "_lib", None)

@@ -52,3 +52,23 @@ def test_pack_int4_roundtrip_all_values():
 def test_bf16_store_is_rne_of_fp32():
     x = np.array([1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, -2.0, 0.0])
     assert synth.store(x, "bf16").tolist() == [0x3F80, 0x3F80, 0x3F82, 0xC000, 0x0000]
+
+
+def test_inputs_match_recorded_digests():
+    """The generator still draws exactly the recorded inputs (digests in
+    tests/golden/synth_sha256.txt, written by make_synth_sha256.py)."""
+    import importlib.util
+    import os
+    golden = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location(
+        "make_synth_sha256", os.path.join(golden, "make_synth_sha256.py"))
+    mk = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mk)
+    recorded = {}
+    with open(os.path.join(golden, "synth_sha256.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                name, d = line.split()
+                recorded[name] = d
+    assert recorded.keys() == mk.CASES.keys()
+    assert mk.compute() == recorded
