@@ -134,6 +134,36 @@ def _empty_out(M, N, tdt, device, pinned=False):
     return t[:, :N]
 
 
+def workload_facts(name, peaks):
+    """Algorithmic work of one launch of a workload and the roofline that
+    bounds it: (flops, alg_bytes, bound, peak, unit).
+
+    flops = 2*M*N*K.  alg_bytes = each operand read once plus C written once:
+    2 or 4 bytes per element, and for the 4-bit path the packed weights
+    (ceil(N/2) bytes per row of K) and the fp16 scales ((K/128) x N).  Padded
+    MMA work and dequantisation arithmetic are not counted.  A contraction
+    whose flops per byte lie below the ridge (tensor peak / HBM bandwidth)
+    is HBM-bound; the fp32 FFMA path is bound by the FMA pipe ("alu"); TF32
+    takes the bf16 peak times the nominal dense ratio 1.1 / 2.25."""
+    base = TRANSPOSED.get(name, (name, False, False))[0]
+    kind, M, N, K = WORKLOADS[base][:4]
+    flops = 2.0 * M * N * K
+    if kind == "w4a16":
+        alg_bytes = M * K * 2 + K * ((N + 1) // 2) + (K // 128) * N * 2 + M * N * 2
+    else:
+        eb = 2 if kind in ("bf16", "f16") else 4
+        alg_bytes = (M * K + K * N + M * N) * eb
+    tensor_peak = peaks["bf16_tflops"]
+    if kind == "f32_tf32":
+        tensor_peak *= 1.1 / 2.25
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if kind == "f32_ffma":
+        return flops, alg_bytes, "alu", ffma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)), "TFLOP/s"
+    if flops / alg_bytes < ridge:
+        return flops, alg_bytes, "hbm", peaks["hbm_gbs"], "GB/s"
+    return flops, alg_bytes, "tensor", tensor_peak, "TFLOP/s"
+
+
 class Case:
     """A workload bound to device buffers, with its roofline facts."""
 
@@ -150,26 +180,21 @@ class Case:
             host["A"] = np.ascontiguousarray(host["A"].T)
         if tb:
             host["B"] = np.ascontiguousarray(host["B"].T)
-        self.flops = 2.0 * M * N * K
+        self.flops, self.alg_bytes, self.bound, self.peak, self.unit = workload_facts(name, peaks)
         if kind == "w4a16":
             self.A = _torch_of(host["A"], "f16", device)
             self.Bq = _torch_of(host["Bq"], "u8", device)
             self.S = _torch_of(host["S"], "f16", device)
             self.C = _empty_out(M, N, torch.float16, device)
-            self.in_bytes = M * K * 2 + host["Bq"].nbytes + host["S"].nbytes
-            self.out_bytes = M * N * 2
             self.dtype = "f16 x int4"
             self._host = host
             self.run = lambda: tg.gemm_w4a16(self.A, self.Bq, self.S, N, C=self.C, relu=relu)
         else:
             ik = {"bf16": "bf16", "f16": "f16"}.get(kind, "f32")
             tdt = {"bf16": torch.bfloat16, "f16": torch.float16}.get(kind, torch.float32)
-            eb = 4 if ik == "f32" else 2
             self.A = _torch_of(host["A"], ik, device)
             self.B = _torch_of(host["B"], ik, device)
             self.C = _empty_out(M, N, tdt, device)
-            self.in_bytes = (M * K + K * N) * eb
-            self.out_bytes = M * N * eb
             self.dtype = {"bf16": "bf16", "f16": "f16", "f32_ffma": "f32", "f32_tf32": "tf32"}[kind]
             self._host = host
             self._ik = ik
@@ -182,19 +207,6 @@ class Case:
             else:
                 mode = tg.F32_TF32 if kind == "f32_tf32" else tg.F32_FFMA
                 self.run = lambda: tg.gemm_f32(self.A, self.B, C=self.C, relu=relu, mode=mode)
-        self.alg_bytes = self.in_bytes + self.out_bytes
-        # roofline bound and peak
-        tensor_peak = peaks["bf16_tflops"]
-        if kind == "f32_tf32":
-            tensor_peak *= 1.1 / 2.25          # nominal tf32 : bf16 dense ratio
-        ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        intensity = self.flops / self.alg_bytes
-        if kind == "f32_ffma":
-            self.bound, self.peak, self.unit = "alu", ffma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)), "TFLOP/s"
-        elif intensity < ridge:
-            self.bound, self.peak, self.unit = "hbm", peaks["hbm_gbs"], "GB/s"
-        else:
-            self.bound, self.peak, self.unit = "tensor", tensor_peak, "TFLOP/s"
 
     def achieved(self, seconds):
         if self.unit == "GB/s":
