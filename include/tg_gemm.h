@@ -203,8 +203,9 @@ TG_API const char *tg_status_string(tg_status s);
 /*
  * tg_last_device_status -- synchronises `stream`, then reads and clears the
  * current device's status word.  Kernels never spin forever: every wait on
- * a pipeline barrier has an iteration limit, and a kernel that hits it
- * records TG_ERR_TIMEOUT there and returns early (C is then incomplete).
+ * a pipeline barrier has a time limit (4 s of device time by default), and a
+ * kernel that hits it records TG_ERR_TIMEOUT there and returns early (C is
+ * then incomplete).
  * Returns TG_OK, TG_ERR_TIMEOUT, or TG_ERR_CUDA if synchronising failed.
  */
 TG_API tg_status tg_last_device_status(void *stream);
