@@ -125,6 +125,46 @@ def test_valid_calls_without_a_device_report_no_device(lib):
     assert _bf16(lib, 8, 8, 0) == NODEV
 
 
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "tg_gemm.h"
+/* Every entry point, called from plain C with arguments that fail
+   validation: prints each status so the test can check them. */
+int main(void) {
+    printf("%d\n", tg_gemm_f32(-1, 8, 8, 0, 8, 0, 8, 0, 8, TG_EPI_NONE, TG_F32_FFMA, 0));
+    printf("%d\n", tg_gemm_f16(8, 8, 8, 0, 8, 0, 8, 0, 8, TG_EPI_NONE, 0));
+    printf("%d\n", tg_gemm_bf16(8, 8, 8, 0, 8, 0, 8, 0, 8, 7, 0));
+    printf("%d\n", tg_gemm_f16_ex(8, 8, 8, 0, 8, 2, 0, 8, 0, 0, 8, TG_EPI_NONE, 0));
+    printf("%d\n", tg_gemm_bf16_ex(8, 8, 8, 0, 8, 0, 0, 8, 3, 0, 8, TG_EPI_NONE, 0));
+    printf("%d\n", tg_gemm_w4a16(4, 32, 256, 0, 256, 0, 16, 0, 32, 64, 0, 32, TG_EPI_NONE, 0));
+    printf("%d\n", tg_gemm_bf16_small_m_static(0, 8, 8, 0, 8, 0, 8, 0, 8, TG_EPI_NONE, 0));
+    printf("%s\n", tg_status_string(TG_ERR_ALIGNMENT));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/tg_gemm.h compiles as strict C99 and a C program links
+    libtg_gemm.so and gets the documented status codes back."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "abi_check.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(binding.lib_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-ltg_gemm",
+                    "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    # negative M; null pointers; bad epilogue; bad trans flags (x2); group 64; M == 0
+    assert out[:7] == [str(c) for c in (INVALID, INVALID, INVALID, INVALID, INVALID, UNSUP, OK)]
+    assert out[7] == "TG_ERR_ALIGNMENT"
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_HERE", str(tmp_path))
     monkeypatch.setattr(binding, "_lib", None)
