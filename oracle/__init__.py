@@ -8,7 +8,9 @@ Each function follows the plain definition of the operation (the scalar
 triple loop on the gtnt.cn TileLang tutorial, section 1.1; C = A x B with
 row-major A and B on the mhpq.cn TileLang GEMM article, section 2.1; the
 ReLU post-processing and the dequantize GEMM on the blog.hotdry.top TileLang
-guide).  The arithmetic lives in ``oracle.c``; this module only marshals
+guide; the FP4-weight GEMM named on the krestaai TileLang architecture page,
+read as MXFP4 weights with bf16 activations).  The arithmetic lives in
+``oracle.c``; this module only marshals
 numpy arrays through ctypes.
 
 Inputs are numpy arrays holding the *stored* values: float32 for fp32,
@@ -44,6 +46,15 @@ def _load():
         lib.oracle_gemm_w4a16.restype = None
         lib.oracle_dequant_w4.argtypes = [i64, i64, vp, i64, vp, i64, i64, dp, i64]
         lib.oracle_dequant_w4.restype = None
+        lib.oracle_gemm_wfp4.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64,
+                                         i64, dp, i64, ctypes.c_int]
+        lib.oracle_gemm_wfp4.restype = None
+        lib.oracle_dequant_fp4.argtypes = [i64, i64, vp, i64, vp, i64, i64, dp, i64]
+        lib.oracle_dequant_fp4.restype = None
+        lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_to_f64.restype = ctypes.c_double
+        lib.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e8m0_to_f64.restype = ctypes.c_double
         lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.oracle_f16_to_f64.restype = ctypes.c_double
         lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -145,6 +156,45 @@ def gemm_w4a16(A_bits, Bq, scales, N, group=128, relu=False):
     _load().oracle_gemm_w4a16(M, N, K, _ptr(A_bits), lda, _ptr(Bq), ldbq,
                               _ptr(scales), lds, group, _ptr(C), N,
                               int(bool(relu)))
+    return C
+
+
+def e2m1_to_f64(code):
+    """Value of one FP4 E2M1 code (0..15)."""
+    return _load().oracle_e2m1_to_f64(int(code))
+
+
+def e8m0_to_f64(e):
+    """Value of one E8M0 scale byte: 2^(e - 127), NaN for 255."""
+    return _load().oracle_e8m0_to_f64(int(e))
+
+
+def dequant_fp4(Bq, scales, N, block=32):
+    """fp64 W (K x N) with W[k, n] = e2m1(code[k, n]) * e8m0(E[k // block, n])."""
+    ldbq = _check2d(Bq, np.uint8, "Bq")
+    lds = _check2d(scales, np.uint8, "scales")
+    K = Bq.shape[0]
+    W = np.empty((K, N), np.float64)
+    _load().oracle_dequant_fp4(K, N, _ptr(Bq), ldbq, _ptr(scales), lds, block,
+                               _ptr(W), N)
+    return W
+
+
+def gemm_wfp4(A_bits, Bq, scales, N, block=32, relu=False):
+    """fp64 value of epi(A . W), W the explicitly dequantised MXFP4 weight.
+
+    A_bits: M x K bf16 bit patterns.  Bq: K x ceil(N/2) bytes of E2M1 codes
+    (low nibble = even column).  scales: (K/block) x N E8M0 bytes.
+    """
+    lda = _check2d(A_bits, np.uint16, "A")
+    ldbq = _check2d(Bq, np.uint8, "Bq")
+    lds = _check2d(scales, np.uint8, "scales")
+    M, K = A_bits.shape
+    if Bq.shape[0] != K:
+        raise ValueError("inner dimensions differ")
+    C = np.empty((M, N), np.float64)
+    _load().oracle_gemm_wfp4(M, N, K, _ptr(A_bits), lda, _ptr(Bq), ldbq,
+                             _ptr(scales), lds, block, _ptr(C), N, int(bool(relu)))
     return C
 
 

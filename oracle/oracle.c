@@ -24,6 +24,14 @@
  *     the library's documented reading: signed 4-bit q packed two per byte,
  *     even column in the low nibble, fp16 scales per 128 rows of K.
  *
+ *   - the FP4-weight ("WFP4") GEMM named in the performance section of
+ *     "TileLang架构深度剖析" (test.krestaai.com.au) likewise multiplies by an
+ *     explicitly dequantised weight.  The pages give no FP4 format; the
+ *     library's reading is MXFP4 from the OCP Microscaling Formats (MX)
+ *     specification v1.0: E2M1 elements (sign, 2 exponent bits with bias 1,
+ *     1 mantissa bit) sharing one E8M0 scale 2^(E - 127) per 32 consecutive
+ *     k of a column, with bf16 activations.
+ *
  * Every stored input value is widened exactly to double, products and sums
  * are taken in double, and ReLU is applied in double.  No blocking, no
  * reordering beyond the i-k-j loop order, no fusion.  Rows of C are spread
@@ -77,6 +85,32 @@ static int oracle_nibble(const uint8_t *row, int64_t n)
     uint8_t byte = row[n >> 1];
     int v = (n & 1) ? (byte >> 4) : (byte & 0x0f);
     return v >= 8 ? v - 16 : v;
+}
+
+/* Unsigned 4-bit code of column n in a packed row (low nibble = even column). */
+static int oracle_code4(const uint8_t *row, int64_t n)
+{
+    uint8_t byte = row[n >> 1];
+    return (n & 1) ? (byte >> 4) : (byte & 0x0f);
+}
+
+/* FP4 E2M1 element -> double (exact).  Bit 3 is the sign, bits 2-1 the
+ * exponent e (bias 1), bit 0 the mantissa m.  e = 0 encodes 0 and the one
+ * subnormal magnitude 0.5 (m * 2^(1-1) / 2); otherwise the value is
+ * 2^(e-1) * (1 + m/2).  The format has no infinity or NaN. */
+double oracle_e2m1_to_f64(uint8_t code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* E8M0 shared scale -> double: 2^(E - 127); E = 255 encodes NaN. */
+double oracle_e8m0_to_f64(uint8_t e)
+{
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -256,6 +290,38 @@ void oracle_gemm_w4a16(int64_t M, int64_t N, int64_t K,
     double *W = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1) * (size_t)(N > 0 ? N : 1));
     oracle_dequant_w4(K, N, Bq, ldbq, scales, lds, group, W, N);
     gemm_generic(M, N, K, A, lda, load_f16, W, N, load_f64, C, ldc, relu);
+    free(W);
+}
+
+/*
+ * Explicit dequantisation of FP4 weights: W[k][n] = e2m1(code[k][n]) *
+ * e8m0(E[k / block][n]), in double (exact: a 2-significant-bit value times a
+ * power of two).  Bq is K rows of ldbq bytes, column n of row k in byte n/2,
+ * low nibble for even n.  scales is (K / block) rows of lds E8M0 bytes.
+ */
+void oracle_dequant_fp4(int64_t K, int64_t N, const uint8_t *Bq, int64_t ldbq,
+                        const uint8_t *scales, int64_t lds, int64_t block,
+                        double *W, int64_t ldw)
+{
+    for (int64_t k = 0; k < K; ++k) {
+        const uint8_t *row = Bq + k * ldbq;
+        const uint8_t *srow = scales + (k / block) * lds;
+        for (int64_t n = 0; n < N; ++n)
+            W[k * ldw + n] = oracle_e2m1_to_f64((uint8_t)oracle_code4(row, n)) *
+                             oracle_e8m0_to_f64(srow[n]);
+    }
+}
+
+/* Dequantise, then the plain GEMM with bf16 activations A (M x K). */
+void oracle_gemm_wfp4(int64_t M, int64_t N, int64_t K,
+                      const uint16_t *A, int64_t lda,
+                      const uint8_t *Bq, int64_t ldbq,
+                      const uint8_t *scales, int64_t lds, int64_t block,
+                      double *C, int64_t ldc, int relu)
+{
+    double *W = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1) * (size_t)(N > 0 ? N : 1));
+    oracle_dequant_fp4(K, N, Bq, ldbq, scales, lds, block, W, N);
+    gemm_generic(M, N, K, A, lda, load_bf16, W, N, load_f64, C, ldc, relu);
     free(W);
 }
 

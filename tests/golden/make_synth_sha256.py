@@ -31,6 +31,8 @@ CASES = {
     "normal_bf16_128x14336x4096_seed3_sqrtk": lambda: synth.normal(128, 14336, 4096, 3, "bf16", True),
     "w4a16_16x8192x8192_seed4": lambda: synth.w4a16(16, 8192, 8192, 4),
     "w4a16_130x300x384_seed4": lambda: synth.w4a16(130, 300, 384, 4),
+    "wfp4_16x8192x8192_seed4": lambda: synth.wfp4(16, 8192, 8192, 4),
+    "wfp4_130x300x384_seed4": lambda: synth.wfp4(130, 300, 384, 4),
 }
 
 

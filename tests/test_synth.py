@@ -72,3 +72,22 @@ def test_inputs_match_recorded_digests():
                 recorded[name] = d
     assert recorded.keys() == mk.CASES.keys()
     assert mk.compute() == recorded
+
+
+def test_pack_nibbles_roundtrip_all_codes():
+    codes = np.arange(16, dtype=np.uint8).reshape(2, 8)
+    packed = synth.pack_nibbles(codes)
+    assert packed.shape == (2, 4)
+    lo, hi = packed & 0xF, packed >> 4
+    assert np.array_equal(lo, codes[:, 0::2]) and np.array_equal(hi, codes[:, 1::2])
+    odd = synth.pack_nibbles(codes[:, :7])          # odd N: zero padding nibble
+    assert odd.shape == (2, 4) and np.all(odd[:, 3] >> 4 == 0)
+
+
+def test_wfp4_inputs():
+    A, Bq, E, codes = synth.wfp4(3, 70, 96, seed=4)
+    assert A.dtype == np.uint16 and A.shape == (3, 96)
+    assert Bq.shape == (96, 35) and E.shape == (3, 70) and codes.shape == (96, 70)
+    assert E.dtype == np.uint8 and E.min() >= 118 and E.max() <= 122
+    assert set(np.unique(codes)) == set(range(16))
+    assert np.array_equal(Bq, synth.pack_nibbles(codes))

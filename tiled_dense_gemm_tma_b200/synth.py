@@ -18,6 +18,8 @@ library's benchmark workloads):
 * fp16 / bf16 matrices are returned as uint16 bit-pattern arrays.
 * The 4-bit weight q (integers in [-8, 7]) is packed two per byte, column
   2j in the low nibble and 2j+1 in the high nibble of byte j of its row.
+  FP4 (E2M1) weight codes 0..15 are packed the same way; their E8M0 scale
+  exponents are stored one byte each.
 """
 import math
 
@@ -50,16 +52,26 @@ def store(x64, dtype):
     raise ValueError(dtype)
 
 
-def pack_int4(q):
-    """Pack an int array (K x N, values in [-8, 7]) into K x ceil(N/2) bytes."""
-    q = np.asarray(q)
-    if q.min(initial=0) < -8 or q.max(initial=0) > 7:
-        raise ValueError("q out of [-8, 7]")
-    K, N = q.shape
-    nib = (q.astype(np.int64) & 0xF).astype(np.uint8)
+def pack_nibbles(codes):
+    """Pack 4-bit codes (K x N, values 0..15) into K x ceil(N/2) bytes:
+    column 2j in the low nibble and 2j+1 in the high nibble of byte j."""
+    c = np.asarray(codes)
+    if c.min(initial=0) < 0 or c.max(initial=0) > 15:
+        raise ValueError("code out of [0, 15]")
+    K, N = c.shape
+    nib = c.astype(np.uint8)
     if N % 2:
         nib = np.concatenate([nib, np.zeros((K, 1), np.uint8)], axis=1)
     return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+
+
+def pack_int4(q):
+    """Pack an int array (K x N, values in [-8, 7]) into K x ceil(N/2) bytes
+    (two's complement nibbles, as pack_nibbles)."""
+    q = np.asarray(q)
+    if q.min(initial=0) < -8 or q.max(initial=0) > 7:
+        raise ValueError("q out of [-8, 7]")
+    return pack_nibbles(q.astype(np.int64) & 0xF)
 
 
 def uniform_pm1(M, N, K, seed, dtype="f32"):
@@ -104,6 +116,26 @@ def w4a16(M, N, K, seed, group=128, s_lo=0.005, s_hi=0.02, a_int=None):
     G = (K + group - 1) // group
     s = rng.uniform(s_lo, s_hi, size=(G, N))
     return store(A, "f16"), pack_int4(q), store(s, "f16"), q
+
+
+def wfp4(M, N, K, seed, block=32, e_lo=118, e_hi=122, a_int=None):
+    """Inputs of the FP4-weight GEMM (MXFP4 weights, bf16 activations).
+
+    Returns (A bf16 bits M x K, Bq packed uint8 K x ceil(N/2) of E2M1 codes,
+    scales uint8 E8M0 exponents ceil(K/block) x N, codes uint8 K x N).  A is
+    N(0, 1), or integers in [-a_int, a_int] when a_int is given; the codes
+    are uniform over all 16 E2M1 codes; the scale exponents are uniform in
+    {e_lo..e_hi} (2^-9 .. 2^-5 by default).
+    """
+    rng = np.random.default_rng(seed)
+    if a_int is None:
+        A = rng.standard_normal(size=(M, K))
+    else:
+        A = rng.integers(-a_int, a_int + 1, size=(M, K)).astype(np.float64)
+    codes = rng.integers(0, 16, size=(K, N)).astype(np.uint8)
+    G = (K + block - 1) // block
+    E = rng.integers(e_lo, e_hi + 1, size=(G, N)).astype(np.uint8)
+    return store(A, "bf16"), pack_nibbles(codes), E, codes
 
 
 def with_ld(X, ld):
