@@ -34,6 +34,13 @@ constexpr int B_STAGE = BK * BN * 4;     // 16 KB
 constexpr int COMPUTE_WARPS = 8;
 constexpr int THREADS = 32 * (COMPUTE_WARPS + 1);
 constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 256 + 1024;
+// Layout guards: the 128-byte-swizzled A stages start on 1024-byte
+// boundaries; the barriers and flags fit their 256 bytes; one CTA fits the
+// 227 KB limit; the 8 compute warps' 8 x 8 register tiles cover the block.
+static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0, "stage alignment");
+static_assert((2 * STAGES + 2) * 8 + 2 * 4 <= 256, "barrier area");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+static_assert(COMPUTE_WARPS * 32 * 64 == BM * BN, "8 x 8 outputs per compute thread");
 
 struct FfmaParams {
     int M, N, K, ldc;

@@ -86,6 +86,15 @@ struct SkCfg {
     static constexpr int SMEM_BYTES = RAW_STAGES * RAW_SLOT + W_STAGES * W_BYTES +
                                       X_STAGES * X_BYTES + 768 + 1024;
     static_assert(MPAD % 16 == 0 && MPAD <= 128, "MPAD");
+    // Layout guards: slots and tiles that hold 128-byte-swizzled boxes start
+    // on 1024-byte boundaries; the ring keeps at least 3 slots in flight; one
+    // CTA fits the 227 KB limit; a 4-bit packed row of a unit is one 128-byte
+    // swizzle span.
+    static_assert(RAW_SLOT % 1024 == 0 && W_BYTES % 1024 == 0 && X_SLICE % 1024 == 0 &&
+                  W_CHUNK % 1024 == 0, "swizzle alignment");
+    static_assert(RAW_STAGES >= 3, "ring");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+    static_assert(!Q4 || GN / 2 == 128, "packed row");
 };
 
 struct SkParams {

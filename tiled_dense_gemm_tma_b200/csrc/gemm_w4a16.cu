@@ -44,6 +44,16 @@ struct W4 {
     static constexpr int SMEM_DATA = RAW_STAGES * (A_BYTES + Q_BYTES) + S_RING +
                                      B_STAGES * B_BYTES + EPI_WARPS * STG_BUF;
     static constexpr int SMEM_BYTES = SMEM_DATA + 256 + 1024;
+    // Layout guards: A, converted B and the staging (128-byte swizzle) and
+    // the packed ring (its TMA boxes) start on 1024-byte boundaries; the
+    // barriers, TMEM slot and abort flag fit their 256 bytes; one CTA fits
+    // the 227 KB limit; the epilogue has one staging buffer per warp.
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0 && B_CHUNK % 1024 == 0, "swizzle");
+    static_assert((RAW_STAGES * A_BYTES + B_STAGES * B_BYTES) % 1024 == 0, "packed ring alignment");
+    static_assert((RAW_STAGES * Q_BYTES) % 1024 == 0 && S_RING % 1024 == 0, "staging alignment");
+    static_assert((2 * RAW_STAGES + 2 * B_STAGES + 5) * 8 + 8 <= 256, "barrier area");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+    static_assert(TMEM_COLS == 512, "TMEM: two 256-column accumulators");
 };
 
 __global__ void __launch_bounds__(W4::THREADS, 1)

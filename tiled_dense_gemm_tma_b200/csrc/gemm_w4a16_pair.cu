@@ -58,6 +58,17 @@ struct W4P {
     static constexpr int SMEM_DATA = STAGES * (A_STAGE + Q_BYTES) + S_RING + B_STAGES * B_STAGE +
                                      EPI_WARPS * 2 * STG_BUF;
     static constexpr int SMEM_BYTES = SMEM_DATA + 512 + 1024;
+    // Layout guards: every 128-byte-swizzled buffer (A, converted B) starts
+    // on a 1024-byte boundary, and so does the packed ring (64-byte swizzle)
+    // and the staging after the scale ring; the barriers, TMEM slot and
+    // abort flag fit their 512 bytes; one CTA fits the 227 KB limit.
+    static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0 && B_CHUNK % 1024 == 0, "swizzle");
+    static_assert((STAGES * A_STAGE + B_STAGES * B_STAGE) % 1024 == 0, "packed ring alignment");
+    static_assert((STAGES * Q_BYTES) % 1024 == 0 && S_RING % 1024 == 0, "staging alignment");
+    static_assert((4 * STAGES + 2 * B_STAGES + 5) * 8 + 8 <= 512, "barrier area");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+    static_assert(TMEM_COLS == 512, "TMEM: two 256-column accumulators");
+    static_assert(32 * CONV_WARPS == 256 && BK * HN / 2 == Q_BYTES, "converter split");
 };
 
 // mbarrier wait with acquire at cluster scope (the arrivals it waits for

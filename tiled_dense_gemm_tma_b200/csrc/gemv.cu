@@ -64,6 +64,19 @@ struct GvCfg {
     static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
     static constexpr int SMEM_BYTES = STAGES * SLOT + RED_BYTES + 512 + 1024;
     static_assert(STAGES >= 3, "ring");
+    // The producer's transaction count is built from these sizes and the
+    // launcher's boxes from GN, BK and MR: each box's bytes must be the
+    // count it is charged.  4-bit: one (GN/2 bytes x BK rows) weight box and
+    // one (GN x 1) fp16 scale box; 16-bit: two (64 x BK) weight boxes; then
+    // KSL (64 x MR) fp16 activation boxes.  A 128-byte-swizzled box is at
+    // most 128 bytes wide and starts on a 1024-byte boundary.
+    static_assert(Q4 ? (W_BYTES == (GN / 2) * BK && GN / 2 == 128)
+                     : (W_BYTES == 2 * W_CHUNK && W_CHUNK == 64 * 2 * BK), "weight box bytes");
+    static_assert(!Q4 || S_BYTES == GN * 2, "scale box bytes");
+    static_assert(X_SLICE == 64 * MR * 2 && X_BYTES == KSL * X_SLICE && KSL * 64 == BK,
+                  "activation box bytes");
+    static_assert(SLOT % 1024 == 0 && W_CHUNK % 1024 == 0, "swizzled boxes on 1024-byte boundaries");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
 
