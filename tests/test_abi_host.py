@@ -105,6 +105,16 @@ def test_row_pitch_limits(lib):
     assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, huge, 0, None) == UNSUP      # ldc
 
 
+def test_ffma_size_limits_refused_before_any_cuda_call(lib):
+    """The fp32 FFMA kernel's own limits (a 32-bit output pitch, at most
+    65535 rows of 128-row tiles) are refused before the library touches
+    CUDA, so they read TG_ERR_UNSUPPORTED even without a device."""
+    f = lib.tg_gemm_f32
+    assert f(8, 8, 8, P, 8, P, 8, P, 1 << 31, 0, 0, None) == UNSUP
+    M = 65535 * 128 + 1
+    assert f(M, 8, 8, P, 8, P, 8, P, 8, 0, 0, None) == UNSUP
+
+
 def test_valid_calls_without_a_device_report_no_device(lib):
     """On a machine with no GPU a well-formed call gets past validation and
     must report TG_ERR_NO_DEVICE (no CPU fallback, no crash).  The fake

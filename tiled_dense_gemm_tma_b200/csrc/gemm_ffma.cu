@@ -285,6 +285,9 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 }  // namespace
 
 int launch_ffma_f32(const GemmArgs& a) {
+    // size limits of this kernel, refused before any CUDA call: a 32-bit
+    // output pitch, and at most 65535 tile rows (grid.y)
+    if (a.ldc > 0x7fffffff || (a.M + BM - 1) / BM > 65535) return kUnsupported;
     int dev = 0;
     if (!current_device(&dev)) return kNoDevice;
     CUtensorMap tA, tB;
@@ -320,9 +323,7 @@ int launch_ffma_f32(const GemmArgs& a) {
     p.status = device_status_ptr();
     p.C = static_cast<float*>(a.C);
     if (!p.status) return kCudaError;
-    if (a.ldc > 0x7fffffff) return kUnsupported;
     dim3 grid(static_cast<unsigned>(tiles_n), static_cast<unsigned>(tiles_m), static_cast<unsigned>(splits));
-    if (grid.y > 65535) return kUnsupported;
     ffma_gemm_kernel<<<grid, THREADS, SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
 }
