@@ -61,6 +61,11 @@ WORKLOADS = {
     "w4a16_gemm_m1": ("w4a16", 1, 8192, 8192, 4, False, "w4a16"),
     "w4a16_gemm_m16": ("w4a16", 16, 8192, 8192, 4, False, "w4a16"),
     "w4a16_gemm_m4096": ("w4a16", 4096, 8192, 8192, 4, False, "w4a16"),
+    # FP4-weight GEMM: bf16 A N(0,1), E2M1 codes uniform over all 16, E8M0
+    # block exponents uniform in {118..122}, the 4-bit workload's shapes
+    "wfp4_gemm_m1": ("wfp4", 1, 8192, 8192, 4, False, "wfp4"),
+    "wfp4_gemm_m16": ("wfp4", 16, 8192, 8192, 4, False, "wfp4"),
+    "wfp4_gemm_m4096": ("wfp4", 4096, 8192, 8192, 4, False, "wfp4"),
 }
 # Transposed-operand variants: name -> (workload, A stored K x M, B stored N x K).
 # The same seeded matrices, stored transposed in HBM.
@@ -95,6 +100,9 @@ def make_inputs(name):
     if kind == "w4a16":
         A, Bq, S, _ = synth.w4a16(M, N, K, seed)
         return {"A": A, "Bq": Bq, "S": S}
+    if kind == "wfp4":
+        A, Bq, E, _ = synth.wfp4(M, N, K, seed)
+        return {"A": A, "Bq": Bq, "S": E}
     st = {"bf16": "bf16", "f16": "f16"}.get(kind, "f32")
     if dist == "normal_sqrtk":
         A, B = synth.normal(M, N, K, seed, st, scale_by_sqrt_k=True)
@@ -139,8 +147,9 @@ def workload_facts(name, peaks):
     bounds it: (flops, alg_bytes, bound, peak, unit).
 
     flops = 2*M*N*K.  alg_bytes = each operand read once plus C written once:
-    2 or 4 bytes per element, and for the 4-bit path the packed weights
-    (ceil(N/2) bytes per row of K) and the fp16 scales ((K/128) x N).  Padded
+    2 or 4 bytes per element, and for the 4-bit paths the packed weights
+    (ceil(N/2) bytes per row of K) and the scales: (K/128) x N fp16, or
+    ceil(K/32) x N E8M0 bytes for FP4 weights.  Padded
     MMA work and dequantisation arithmetic are not counted.  A contraction
     whose flops per byte lie below the ridge (tensor peak / HBM bandwidth)
     is HBM-bound; the fp32 FFMA path is bound by the FMA pipe ("alu"); TF32
@@ -150,6 +159,8 @@ def workload_facts(name, peaks):
     flops = 2.0 * M * N * K
     if kind == "w4a16":
         alg_bytes = M * K * 2 + K * ((N + 1) // 2) + (K // 128) * N * 2 + M * N * 2
+    elif kind == "wfp4":
+        alg_bytes = M * K * 2 + K * ((N + 1) // 2) + ((K + 31) // 32) * N + M * N * 2
     else:
         eb = 2 if kind in ("bf16", "f16") else 4
         alg_bytes = (M * K + K * N + M * N) * eb
@@ -189,6 +200,14 @@ class Case:
             self.dtype = "f16 x int4"
             self._host = host
             self.run = lambda: tg.gemm_w4a16(self.A, self.Bq, self.S, N, C=self.C, relu=relu)
+        elif kind == "wfp4":
+            self.A = _torch_of(host["A"], "bf16", device)
+            self.Bq = _torch_of(host["Bq"], "u8", device)
+            self.S = _torch_of(host["S"], "u8", device)
+            self.C = _empty_out(M, N, torch.bfloat16, device)
+            self.dtype = "bf16 x fp4 (e2m1, e8m0 per 32 k)"
+            self._host = host
+            self.run = lambda: tg.gemm_wfp4(self.A, self.Bq, self.S, N, C=self.C, relu=relu)
         else:
             ik = {"bf16": "bf16", "f16": "f16"}.get(kind, "f32")
             tdt = {"bf16": torch.bfloat16, "f16": torch.float16}.get(kind, torch.float32)
@@ -216,10 +235,11 @@ class Case:
     def host_pinned(self):
         """Pinned host copies of the inputs and a pinned host output (e2e)."""
         import torch
-        if self.kind == "w4a16":
-            hA = _torch_of(self._host["A"], "f16", "cpu", pinned=True)
+        if self.kind in ("w4a16", "wfp4"):
+            ak, sk = ("f16", "f16") if self.kind == "w4a16" else ("bf16", "u8")
+            hA = _torch_of(self._host["A"], ak, "cpu", pinned=True)
             hB = _torch_of(self._host["Bq"], "u8", "cpu", pinned=True)
-            hS = _torch_of(self._host["S"], "f16", "cpu", pinned=True)
+            hS = _torch_of(self._host["S"], sk, "cpu", pinned=True)
             return [(self.A, hA), (self.Bq, hB), (self.S, hS)], \
                 _empty_out(self.M, self.N, self.C.dtype, "cpu", pinned=True)
         hA = _torch_of(self._host["A"], self._ik, "cpu", pinned=True)
@@ -233,13 +253,16 @@ class Case:
 class ClockSampler:
     """Samples the GPU's SM clock, power and clock-event reasons while the
     timed region runs.  Read-only NVML queries from a background thread every
-    20 ms; the GPU is found by the CUDA device's PCI address, so the sampled
-    GPU is the one the bench runs on whatever the visible-device mapping.
-    Falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
+    millisecond, each sample stamped with the host clock; the GPU is found by
+    the CUDA device's PCI address, so the sampled GPU is the one the bench
+    runs on whatever the visible-device mapping.  summary() reports the
+    samples taken between the host times that bracket the timed region (the
+    GPU runs the region's launches between them).  Falls back to
+    `nvidia-smi -lms 100` when NVML is unavailable."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    PERIOD_S = 0.02
+    PERIOD_S = 0.001
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
@@ -269,7 +292,8 @@ class ClockSampler:
                 pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
                 self.rows.append(["0", str(sm), str(mx), str(pw), hex(r)] +
-                                 ["Active" if r & b else "Not Active" for b in bits])
+                                 ["Active" if r & b else "Not Active" for b in bits] +
+                                 [time.time()])
             except Exception:                        # stop sampling, keep what we have
                 return
             time.sleep(self.PERIOD_S)
@@ -312,8 +336,17 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, window=None):
+        """Clock record; with window = (t0, t1) host times, only the samples
+        taken inside it (all samples when none fell inside)."""
         rows = list(self.rows)
+        in_window = None
+        if window is not None:
+            t0, t1 = window
+            inside = [r for r in rows if len(r) > 9 and t0 <= r[9] <= t1]
+            in_window = len(inside)
+            if inside:
+                rows = inside
         if self.path and os.path.exists(self.path):
             with open(self.path) as f:
                 for line in f:
@@ -338,9 +371,11 @@ class ClockSampler:
         # samples under load: power well above idle
         loaded = [s for s, p in zip(sm, pw) if p is not None and pw and p > 0.5 * max(pw)] or sm
         return {"sm_mhz": float(np.median(loaded)) if loaded else None,
+                "sm_mhz_mean": round(float(np.mean(loaded)), 1) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None,
                 "power_w_max": max(pw) if pw else None,
-                "samples": len(rows), "reasons": reasons}
+                "samples": len(rows), "samples_in_timed_region": in_window,
+                "period_ms": self.PERIOD_S * 1e3, "reasons": reasons}
 
 
 def flush_l2(bufs):
@@ -408,14 +443,15 @@ def oracle_block(name, host, rows, cols):
     """Run the fp64 oracle on the block C[rows, cols] (full K); return seconds."""
     import oracle
     kind = WORKLOADS[name][0]
-    if kind == "w4a16":
+    if kind in ("w4a16", "wfp4"):
         A = np.ascontiguousarray(host["A"][rows])
         ncols = len(cols)
         c0 = int(cols[0]) & ~1
         Bq = np.ascontiguousarray(host["Bq"][:, c0 // 2:(c0 + ncols + 1) // 2 + 1])
         S = np.ascontiguousarray(host["S"][:, c0:c0 + ncols])
+        fn = oracle.gemm_w4a16 if kind == "w4a16" else oracle.gemm_wfp4
         t0 = time.perf_counter()
-        oracle.gemm_w4a16(A, Bq, S, N=ncols)
+        fn(A, Bq, S, N=ncols)
         return time.perf_counter() - t0
     A = np.ascontiguousarray(host["A"][rows])
     B = np.ascontiguousarray(host["B"][:, cols])
@@ -569,6 +605,7 @@ def main():
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize()
+        h0 = time.time()
         t_start.record()
         for i in range(K):
             ev_s[i].record()
@@ -576,8 +613,9 @@ def main():
             ev_e[i].record()
         t_end.record()
         torch.cuda.synchronize()
+        h1 = time.time()
         barrier()
-    clocks = clk.summary()
+    clocks = clk.summary(window=(h0, h1))
     elapsed = max_over_ranks(group, t_start.elapsed_time(t_end) * 1e-3, dev)
     launch_s = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_s, ev_e)])) * 1e-3
     st = tg.last_device_status()
@@ -665,6 +703,7 @@ def main():
             "roofline": {"bound": case.bound, "achieved": round(achieved, 2),
                          "peak": case.peak, "unit": case.unit,
                          "frac": round(achieved / case.peak, 4),
+                         "sm_mhz_mean": clocks.get("sm_mhz_mean"),
                          "traffic": traffic, "peak_source": f"{peak_src} (burst)",
                          "peak_sustained": sustained,
                          "frac_of_sustained": (round(achieved / sustained, 4) if sustained else None),

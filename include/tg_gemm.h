@@ -21,8 +21,8 @@
  * - Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
  *   current CUDA device.  The caller owns every buffer.  C must not overlap
  *   A, B or the scales (not checked).
- * - Leading dimensions are in elements (in bytes for the packed 4-bit
- *   weight), and must be >= the row length.
+ * - Leading dimensions are in elements (in bytes for packed 4-bit weights
+ *   and E8M0 scale bytes), and must be >= the row length.
  * - stream is a cudaStream_t passed as void*; NULL means the legacy default
  *   stream.  Calls are asynchronous: they validate, enqueue and return.
  * - Sizes: M, N, K >= 0.  M == 0 or N == 0 -> TG_OK, nothing is launched.
@@ -70,7 +70,8 @@ typedef enum {
     TG_OK = 0,
     TG_ERR_INVALID_ARG = 1,  /* negative size, NULL pointer, ld < row length, bad flag */
     TG_ERR_ALIGNMENT = 2,    /* base not 16-byte aligned or row pitch not a multiple of 16 bytes */
-    TG_ERR_UNSUPPORTED = 3,  /* group size other than 128, K not a multiple of it, size limit */
+    TG_ERR_UNSUPPORTED = 3,  /* 4-bit group / block size other than 128 / 32, K not a multiple of
+                                the group, size limit */
     TG_ERR_CUDA = 4,         /* a CUDA runtime / driver call or the launch failed */
     TG_ERR_TIMEOUT = 5,      /* a kernel's bounded wait expired (reported by tg_last_device_status) */
     TG_ERR_NO_DEVICE = 6     /* no sm_100 device is current */
@@ -129,10 +130,11 @@ TG_API tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
  *   trans_b = 0: B is K x N, row pitch ldb >= N;  trans_b = 1: B is stored
  *                N x K (op(B) = B^T), row pitch ldb >= K.
  * trans flags other than 0 / 1 -> TG_ERR_INVALID_ARG.  With both flags 0
- * this is tg_gemm_f16 / tg_gemm_bf16.  A transposed call always runs the
- * CTA-pair tensor-core kernel (no small-M variant), and returns
- * TG_ERR_UNSUPPORTED if the device refuses its cluster launch.  Same
- * alignment, status and ownership rules as tg_gemm_f16.
+ * this is tg_gemm_f16 / tg_gemm_bf16.  A call with only B transposed and
+ * M <= 128 runs the weight-streaming small-M kernel on K-major weight
+ * tiles; every other transposed call runs the CTA-pair tensor-core kernel
+ * and returns TG_ERR_UNSUPPORTED if the device refuses its cluster launch.
+ * Same alignment, status and ownership rules as tg_gemm_f16.
  */
 TG_API tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K,
                          const void *A, int64_t lda, int trans_a,
@@ -172,6 +174,37 @@ TG_API tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
                         const void *scales, int64_t lds, int group_size,
                         void *C, int64_t ldc,
                         int epilogue, void *stream);
+
+/*
+ * tg_gemm_wfp4 -- FP4-weight GEMM ("WFP4", the low-precision GEMM of the
+ * performance section, 性能表现与基准测试验证, of "TileLang架构深度剖析"
+ * (test.krestaai.com.au); the pages give no format, this library reads it
+ * as the MXFP4 weights of the OCP Microscaling Formats (MX) specification
+ * v1.0 with bf16 activations):  C = epi(A . W) with
+ *
+ *     W[k][n] = e2m1(code[k][n]) * 2^(E[k / 32][n] - 127)
+ *
+ *   A:      M x K bf16 activations, row pitch lda (elements, % 8 == 0)
+ *   Bq:     K rows of E2M1 codes, two per byte: column 2j in bits 0-3 and
+ *           column 2j+1 in bits 4-7 of byte j.  A code is a sign (bit 3), a
+ *           2-bit exponent with bias 1 (bits 2-1) and a mantissa bit (bit 0):
+ *           magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.  Row pitch ldbq in BYTES
+ *           (>= ceil(N/2), % 16 == 0).
+ *   scales: ceil(K / 32) x N E8M0 bytes E (the scale 2^(E - 127); E = 255
+ *           means NaN), row pitch lds in BYTES (>= N, % 16 == 0).
+ *   block_size: must be 32 (k rows per scale), else TG_ERR_UNSUPPORTED.
+ *   C:      M x N bf16 output, row pitch ldc (elements, % 8 == 0).
+ * Any K >= 0.  W is formed exactly as a bf16 tensor-core operand (for
+ * E <= 252; a larger E overflows bf16), products accumulate in fp32, and the
+ * result is rounded once to bf16.  Same status and ownership rules as
+ * tg_gemm_w4a16.
+ */
+TG_API tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K,
+                       const void *A, int64_t lda,
+                       const uint8_t *Bq, int64_t ldbq,
+                       const uint8_t *scales, int64_t lds, int block_size,
+                       void *C, int64_t ldc,
+                       int epilogue, void *stream);
 
 /*
  * tg_gemm_bf16_small_m_static -- tg_gemm_bf16 for M <= 128 that never

@@ -86,6 +86,23 @@ def test_argument_validation_w4a16(lib):
     assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 3, None) == INVALID
 
 
+def test_argument_validation_wfp4(lib):
+    w = lib.tg_gemm_wfp4
+    # M, N, K, A, lda, Bq, ldbq, scales, lds (bytes), block, C, ldc, epi, stream
+    assert w(4, 32, 256, P, 256, P, 16, P, 32, 16, P, 32, 0, None) == UNSUP     # block 16
+    assert w(4, 32, 256, P, 256, P, 8, P, 32, 32, P, 32, 0, None) == INVALID    # ldbq < N/2
+    assert w(4, 32, 256, P, 256, P, 16, P, 16, 32, P, 32, 0, None) == INVALID   # lds < N bytes
+    assert w(4, 32, 256, P, 256, P, 24, P, 32, 32, P, 32, 0, None) == ALIGN     # ldbq % 16
+    assert w(4, 40, 256, P, 256, P, 32, P, 40, 32, P, 40, 0, None) == ALIGN     # lds % 16
+    assert w(4, 32, 256, P, 256, P, 16, P + 8, 32, 32, P, 32, 0, None) == ALIGN
+    assert w(4, 32, 256, P, 256, P, 16, None, 32, 32, P, 32, 0, None) == INVALID
+    assert w(0, 32, 256, P, 256, P, 16, P, 32, 32, P, 32, 0, None) == OK
+    assert w(4, 32, 256, P, 256, P, 16, P, 32, 32, P, 32, 2, None) == INVALID
+    huge = (1 << 62) + 8
+    assert w(4, 32, 256, P, 256, P, 16, P, huge, 32, P, 32, 0, None) == UNSUP   # lds
+    assert w(4, 32, 256, P, 256, P, 1 << 40, P, 32, 32, P, 32, 0, None) == UNSUP
+
+
 def test_row_pitch_limits(lib):
     """Row pitches of 2^40 bytes or more are refused before any product
     ld * sizeof(element) is formed, so even pitches near 2^63 are reported
@@ -103,6 +120,26 @@ def test_row_pitch_limits(lib):
     assert w(4, 32, 256, P, 256, P, 16, P, huge, 128, P, 32, 0, None) == UNSUP      # lds
     assert w(4, 32, 256, P, huge, P, 16, P, 32, 128, P, 32, 0, None) == UNSUP       # lda
     assert w(4, 32, 256, P, 256, P, 16, P, 32, 128, P, huge, 0, None) == UNSUP      # ldc
+    s = lib.tg_gemm_bf16_small_m_static
+    for big in (1 << 40, huge):
+        assert s(16, 8, 8, P, big, P, 8, P, 8, 0, None) == UNSUP                    # lda
+        assert s(16, 8, 8, P, 8, P, big, P, 8, 0, None) == UNSUP                    # ldb
+        assert s(16, 8, 8, P, 8, P, 8, P, big, 0, None) == UNSUP                    # ldc
+
+
+def test_argument_validation_small_m_static(lib):
+    """The entry point that never allocates runs the same checks as
+    tg_gemm_bf16 before any CUDA call, plus its own M <= 128 limit."""
+    s = lib.tg_gemm_bf16_small_m_static
+    assert s(-1, 8, 8, P, 8, P, 8, P, 8, 0, None) == INVALID
+    assert s(16, 8, 8, P, 8, P, 8, P, 8, 2, None) == INVALID            # bad epilogue
+    assert s(16, 8, 8, None, 8, P, 8, P, 8, 0, None) == INVALID
+    assert s(16, 8, 8, P, 7, P, 8, P, 8, 0, None) == INVALID            # lda < K
+    assert s(16, 8, 8, P + 8, 8, P, 8, P, 8, 0, None) == ALIGN
+    assert s(16, 8, 8, P, 12, P, 8, P, 8, 0, None) == ALIGN             # 24-byte pitch
+    assert s(0, 8, 8, P, 8, P, 8, P, 8, 0, None) == OK
+    assert s(129, 8, 8, P, 8, P, 8, P, 8, 0, None) == UNSUP             # M above 128
+    assert s(16, 1 << 31, 8, P, 8, P, 1 << 31, P, 1 << 31, 0, None) == UNSUP
 
 
 def test_ffma_size_limits_refused_before_any_cuda_call(lib):
@@ -128,6 +165,7 @@ def test_valid_calls_without_a_device_report_no_device(lib):
     for mode in (0, 1):
         assert lib.tg_gemm_f32(64, 64, 64, P, 64, P, 64, P, 64, 0, mode, None) == NODEV
     assert lib.tg_gemm_w4a16(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 0, None) == NODEV
+    assert lib.tg_gemm_wfp4(4, 32, 200, P, 200, P, 16, P, 32, 32, P, 32, 0, None) == NODEV
     assert lib.tg_gemm_bf16_ex(64, 64, 64, P, 64, 1, P, 64, 1, P, 64, 0, None) == NODEV
     assert lib.tg_gemm_f16_ex(64, 64, 64, P, 64, 0, P, 64, 1, P, 64, 0, None) == NODEV
     assert lib.tg_gemm_bf16_small_m_static(16, 64, 64, P, 64, P, 64, P, 64, 0, None) == NODEV
@@ -148,6 +186,7 @@ int main(void) {
     printf("%d\n", tg_gemm_bf16_ex(8, 8, 8, 0, 8, 0, 0, 8, 3, 0, 8, TG_EPI_NONE, 0));
     printf("%d\n", tg_gemm_w4a16(4, 32, 256, 0, 256, 0, 16, 0, 32, 64, 0, 32, TG_EPI_NONE, 0));
     printf("%d\n", tg_gemm_bf16_small_m_static(0, 8, 8, 0, 8, 0, 8, 0, 8, TG_EPI_NONE, 0));
+    printf("%d\n", tg_gemm_wfp4(4, 32, 256, 0, 256, 0, 16, 0, 32, 16, 0, 32, TG_EPI_NONE, 0));
     printf("%s\n", tg_status_string(TG_ERR_ALIGNMENT));
     return 0;
 }
@@ -170,9 +209,11 @@ def test_header_is_plain_c_and_links(tmp_path):
                     "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-ltg_gemm",
                     "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
-    # negative M; null pointers; bad epilogue; bad trans flags (x2); group 64; M == 0
-    assert out[:7] == [str(c) for c in (INVALID, INVALID, INVALID, INVALID, INVALID, UNSUP, OK)]
-    assert out[7] == "TG_ERR_ALIGNMENT"
+    # negative M; null pointers; bad epilogue; bad trans flags (x2); group 64; M == 0;
+    # FP4 block 16
+    assert out[:8] == [str(c) for c in (INVALID, INVALID, INVALID, INVALID, INVALID, UNSUP, OK,
+                                        UNSUP)]
+    assert out[8] == "TG_ERR_ALIGNMENT"
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -39,6 +39,10 @@ EXPECTED = {
     "w4a16_gemm_m1": (0.1342, 34.62, "hbm"),
     "w4a16_gemm_m16": (2.147, 35.13, "hbm"),
     "w4a16_gemm_m4096": (549.8, 168.8, "tensor"),
+    # FP4 weights: 33.55 MB codes + 2.10 MB E8M0 bytes (one per 32 k per column)
+    "wfp4_gemm_m1": (0.1342, 35.68, "hbm"),
+    "wfp4_gemm_m16": (2.147, 36.18, "hbm"),
+    "wfp4_gemm_m4096": (549.8, 169.9, "tensor"),
 }
 
 
@@ -74,6 +78,13 @@ def test_packed_weight_bytes_match_the_generator():
     kind, M, N, K = bench.WORKLOADS["w4a16_gemm_m1"][:4]
     nbytes = host["A"].nbytes + host["Bq"].nbytes + host["S"].nbytes + M * N * 2
     assert bench.workload_facts("w4a16_gemm_m1", PEAKS)[1] == nbytes
+
+
+def test_fp4_weight_bytes_match_the_generator():
+    host = bench.make_inputs("wfp4_gemm_m16")
+    kind, M, N, K = bench.WORKLOADS["wfp4_gemm_m16"][:4]
+    nbytes = host["A"].nbytes + host["Bq"].nbytes + host["S"].nbytes + M * N * 2
+    assert bench.workload_facts("wfp4_gemm_m16", PEAKS)[1] == nbytes
 
 
 def test_traffic_record_follows_the_source_digest(monkeypatch):

@@ -57,6 +57,33 @@ class FakeLib:
         return 0
 
 
+def _read_bytes(ptr, rows, cols, ld, dtype):
+    """rows x cols array of `dtype` at host address ptr, row pitch ld elements."""
+    if rows == 0 or cols == 0:
+        return np.zeros((rows, cols), dtype)
+    ct = ctypes.c_uint16 if dtype == np.uint16 else ctypes.c_uint8
+    n = (rows - 1) * ld + cols
+    raw = np.ctypeslib.as_array((ct * n).from_address(ptr)).astype(dtype)
+    u = np.zeros(rows * ld, dtype)
+    u[:n] = raw
+    return np.ascontiguousarray(u.reshape(rows, ld)[:, :cols])
+
+
+def _fake_wfp4(self, M, N, K, A, lda, Bq, ldbq, S, lds, block, C, ldc, epi, stream):
+    """Reads the FP4-weight operands back through the pointers and pitches it
+    is given and multiplies them with the oracle."""
+    import oracle
+    self.calls.append(dict(kind="wfp4", M=M, N=N, K=K, lda=lda, ldbq=ldbq, lds=lds, block=block))
+    a = _read_bytes(A, M, K, lda, np.uint16)
+    q = _read_bytes(Bq, K, (N + 1) // 2, ldbq, np.uint8)
+    e = _read_bytes(S, (K + block - 1) // block, N, lds, np.uint8)
+    _write(C, M, N, ldc, oracle.gemm_wfp4(a, q, e, N=N, block=block, relu=epi == 1))
+    return 0
+
+
+FakeLib.tg_gemm_wfp4 = _fake_wfp4
+
+
 @pytest.fixture
 def fake(monkeypatch):
     lib = FakeLib()
@@ -145,3 +172,30 @@ def test_operands_must_be_cuda_tensors():
     s = torch.zeros(1, 16, dtype=torch.float16)
     with pytest.raises(ValueError, match="CUDA"):
         binding.gemm_w4a16(torch.zeros(4, 128, dtype=torch.float16), q, s, 16)
+
+
+def test_wfp4_marshalling(fake):
+    """gemm_wfp4 passes the activations, packed codes and scale bytes with
+    their own pitches (elements for A, bytes for the packed codes and the
+    E8M0 rows) and the block size; a wider-than-needed pitch on each operand
+    makes a mix-up visible."""
+    import oracle
+    from tiled_dense_gemm_tma_b200 import synth
+    M, N, K = 5, 40, 96
+    A, Bq, E, _ = synth.wfp4(M, N, K, seed=3)
+    tA = torch.zeros((M, K + 8), dtype=torch.int16)
+    tA[:, :K] = torch.from_numpy(A.view(np.int16))
+    tA = tA.view(torch.bfloat16)[:, :K]
+    tq = torch.zeros((K, 48), dtype=torch.uint8)
+    tq[:, :Bq.shape[1]] = torch.from_numpy(Bq)
+    te = torch.zeros((E.shape[0], 64), dtype=torch.uint8)
+    te[:, :N] = torch.from_numpy(E)
+    te = te[:, :N]
+    C = binding.gemm_wfp4(tA, tq, te, N, relu=True)
+    call = fake.calls[-1]
+    assert (call["M"], call["N"], call["K"], call["block"]) == (M, N, K, 32)
+    assert (call["lda"], call["ldbq"], call["lds"]) == (K + 8, 48, 64)
+    ref = oracle.gemm_wfp4(A, Bq, E, N=N, relu=True)
+    _close(C, torch.from_numpy(ref))
+    with pytest.raises(TypeError):
+        binding.gemm_wfp4(tA.view(torch.float16), tq, te, N)

@@ -1,8 +1,9 @@
 """The one-CTA tensor-core kernels are the fallback when a cluster (CTA-pair)
 launch is refused.  TG_NO_PAIR=1 makes every pair launch report
 "unsupported" (read once per process, so the check runs in a child
-process); bf16, fp16 and w4a16 GEMMs with M > 128 must then still match the
-fp64 oracle at rtol = atol = 1e-2.
+process); bf16, fp16, w4a16 and FP4-weight GEMMs with M > 128 must then still match the
+fp64 oracle at rtol = atol = 1e-2, on shapes with one tile per CTA and with
+more tiles than CTAs.
 """
 import os
 import subprocess
@@ -29,10 +30,24 @@ CHILD = textwrap.dedent("""
         C = fn(to_dev(A, kind), to_dev(B, kind), relu=True)
         ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B, True)
         assert_close(decode16(from_dev(C, kind), kind), ref, 1e-2, 1e-2, kind)
-    A, Bq, S, _ = synth.w4a16(257, 520, 384, seed=4)
-    C = tg.gemm_w4a16(to_dev(A, "f16"), to_dev(Bq, "u8"), to_dev(S, "f16"), 520)
-    assert_close(decode16(from_dev(C, "f16"), "f16"), oracle.gemm_w4a16(A, Bq, S, N=520),
-                 1e-2, 1e-2, "w4a16")
+    # 16 x 11 = 176 tiles of 128 x 256 for 148 persistent CTAs: CTAs run a
+    # second tile (accumulator double buffer, ring phases across tiles)
+    for kind in ("bf16", "f16"):
+        A, B = synth.normal(2000, 2600, 320, seed=2, dtype=kind, scale_by_sqrt_k=True)
+        fn = tg.gemm_bf16 if kind == "bf16" else tg.gemm_f16
+        C = fn(to_dev(A, kind), to_dev(B, kind))
+        ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B)
+        assert_close(decode16(from_dev(C, kind), kind), ref, 1e-2, 1e-2, kind + " many tiles")
+    for (M, N, K) in ((257, 520, 384), (2048, 2600, 512)):
+        A, Bq, S, _ = synth.w4a16(M, N, K, seed=4)
+        C = tg.gemm_w4a16(to_dev(A, "f16"), to_dev(Bq, "u8"), to_dev(S, "f16"), N)
+        assert_close(decode16(from_dev(C, "f16"), "f16"), oracle.gemm_w4a16(A, Bq, S, N=N),
+                     1e-2, 1e-2, f"w4a16 {M}x{N}x{K}")
+    for (M, N, K) in ((257, 520, 384), (2048, 2600, 480)):
+        A, Bq, E, _ = synth.wfp4(M, N, K, seed=4)
+        C = tg.gemm_wfp4(to_dev(A, "bf16"), to_dev(Bq, "u8"), to_dev(E, "u8"), N)
+        assert_close(decode16(from_dev(C, "bf16"), "bf16"), oracle.gemm_wfp4(A, Bq, E, N=N),
+                     1e-2, 1e-2, f"wfp4 {M}x{N}x{K}")
     torch.cuda.synchronize()
     print("RESULT", tg.last_device_status())
 """) % (ROOT, os.path.join(ROOT, "tests"))

@@ -119,13 +119,19 @@ def _sampled_check(tg, kind, M, N, K, seed, relu=False, nsamp=48):
     assert_close(got[rows], ref_rows, RTOL, ATOL, f"{kind} rows")
     ref_cols = _oracle16(kind, A, np.ascontiguousarray(B[:, cols]), relu)
     assert_close(got[:, cols], ref_cols, RTOL, ATOL, f"{kind} cols")
+    # the relative Frobenius gate is the sharp one (|C| ~ 1e-2 with these
+    # entries): it covers every sampled row and every sampled column
     assert rel_frob(got[rows], ref_rows) <= FROB[kind]
+    assert rel_frob(got[:, cols], ref_cols) <= FROB[kind]
+    if relu:
+        assert np.all(got[rows] >= 0) and np.all(got[:, cols] >= 0)
 
 
 @pytest.mark.parametrize("kind", ["bf16", "f16"])
 @pytest.mark.parametrize("size", [4096, 8192])
-def test_full_size_square_sampled(tg, kind, size):
-    _sampled_check(tg, kind, size, size, size, seed=2, relu=(size == 4096))
+@pytest.mark.parametrize("relu", [False, True])
+def test_full_size_square_sampled(tg, kind, size, relu):
+    _sampled_check(tg, kind, size, size, size, seed=2, relu=relu)
 
 
 @pytest.mark.parametrize("shape", [(8192, 1024, 8192), (3000, 5000, 4000), (128, 14336, 4096),
@@ -156,6 +162,48 @@ def test_tf32_random(tg, shape):
     got = _run_f32(tg, A, B, tg.F32_TF32)
     ref = oracle.gemm_f32(A, B)
     assert rel_frob(got, ref) <= 5e-3
+
+
+def test_tf32_full_1024(tg):
+    # the TF32 configuration at 1024^3, every output against the oracle
+    A, B = synth.normal(1024, 1024, 1024, seed=1)
+    got = _run_f32(tg, A, B, tg.F32_TF32)
+    assert rel_frob(got, oracle.gemm_f32(A, B)) <= 5e-3
+
+
+def test_tf32_many_tiles_per_cta(tg):
+    # 16 x 29 = 464 tiles of 128 x 256 for 148 persistent CTAs (> 3 per CTA):
+    # every CTA wraps both TMEM accumulator buffers and the ring phases
+    # several times; ragged N and K
+    M, N, K = 2048, 7400, 100
+    A, B = synth.normal(M, N, K, seed=1)
+    for relu in (False, True):
+        got = _run_f32(tg, A, B, tg.F32_TF32, relu=relu)
+        assert rel_frob(got, oracle.gemm_f32(A, B, relu)) <= 5e-3
+
+
+@pytest.mark.parametrize("kind", ["normal", "integer"])
+def test_tf32_full_size_4096_sampled(tg, kind):
+    # the TF32 configuration at 4096^3 (512 tiles): sampled full rows and
+    # columns; integer data {-3..3} is exact in TF32 and fp32, so bit-exact
+    import torch
+    n = 4096
+    A, B = synth.normal(n, n, n, seed=1) if kind == "normal" else synth.integers(n, n, n, seed=1)
+    C = tg.gemm_f32(to_dev(A, "f32"), to_dev(B, "f32"), mode=tg.F32_TF32)
+    torch.cuda.synchronize()
+    assert tg.last_device_status() == 0
+    got = from_dev(C, "f32")
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.concatenate([[0, n - 1], rng.choice(n, 40, replace=False)]))
+    cols = np.unique(np.concatenate([[0, n - 1], rng.choice(n, 40, replace=False)]))
+    ref_r = oracle.gemm_f32(np.ascontiguousarray(A[rows]), B)
+    ref_c = oracle.gemm_f32(A, np.ascontiguousarray(B[:, cols]))
+    if kind == "integer":
+        assert np.array_equal(got[rows], oracle.round_f32(ref_r))
+        assert np.array_equal(got[:, cols], oracle.round_f32(ref_c))
+    else:
+        assert rel_frob(got[rows], ref_r) <= 5e-3
+        assert rel_frob(got[:, cols], ref_c) <= 5e-3
 
 
 def test_tf32_integer_bit_exact(tg):

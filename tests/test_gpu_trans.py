@@ -5,7 +5,9 @@ on them (dA = dC . B^T, dB = A^T . dC), against the fp64 oracle.
 The oracle multiplies the logical (untransposed) matrices; the GPU reads the
 stored transposes.  Tolerance rtol = atol = 1e-2 as for the plain 16-bit
 GEMM; integer data in {-1, 0, 1} must match bit-exactly.  Shapes include
-ragged edges in every dimension and M below the 256-row pair tile.
+ragged edges in every dimension, M below the 256-row pair tile, more pair
+tiles than CTA pairs, and small M with B transposed (the weight-streaming
+kernel on K-major weight tiles).
 """
 import numpy as np
 import pytest
@@ -61,6 +63,52 @@ def test_transposed_operands(tg, kind, shape, trans):
         ref = ref_fn(A, B, relu)
         assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} {trans} relu={relu}")
         assert rel_frob(got, ref) <= FROB[kind]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+@pytest.mark.parametrize("trans", TRANS)
+def test_transposed_many_tiles_per_pair(tg, kind, trans):
+    # 16 x 11 = 176 pair tiles of 256 x 256 for 74 CTA pairs: every pair runs
+    # two or three tiles, wrapping its TMEM accumulators and ring phases
+    # across tiles; ragged in M, N and K
+    M, N, K = 4000, 2600, 650
+    A, B = synth.normal(M, N, K, seed=2, dtype=kind, scale_by_sqrt_k=True)
+    got = decode16(_run(tg, kind, A, B, *trans), kind)
+    ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B)
+    assert_close(got, ref, RTOL, ATOL, f"{kind} {trans}")
+    assert rel_frob(got, ref) <= FROB[kind]
+
+
+SMALL_M_TB = [(1, 8192, 8192), (3, 1000, 700), (16, 8192, 8192), (17, 520, 333),
+              (100, 777, 1200), (128, 14336, 4096), (64, 130, 72)]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+@pytest.mark.parametrize("shape", SMALL_M_TB)
+def test_small_m_transposed_b(tg, kind, shape):
+    # B stored N x K with M <= 128 (the backward product dA = dC . B^T at
+    # small batch): the weight-streaming kernel reads K-major weight tiles
+    M, N, K = shape
+    A, B = synth.normal(M, N, K, seed=3, dtype=kind, scale_by_sqrt_k=True)
+    ref_fn = oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16
+    for relu in (False, True):
+        got = decode16(_run(tg, kind, A, B, False, True, relu=relu), kind)
+        ref = ref_fn(A, B, relu)
+        assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} relu={relu}")
+        assert rel_frob(got, ref) <= FROB[kind]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+def test_small_m_transposed_b_bit_exact_and_repeatable(tg, kind):
+    M, N, K = 24, 1536, 256
+    A, B = synth.integers(M, N, K, seed=1, lo=-1, hi=1, dtype=kind)
+    ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B)
+    rnd = oracle.round_bf16(ref) if kind == "bf16" else oracle.round_f16(ref)
+    assert np.array_equal(decode16(_run(tg, kind, A, B, False, True), kind), decode16(rnd, kind))
+    A, B = synth.normal(16, 4096, 8192, seed=3, dtype=kind, scale_by_sqrt_k=True)
+    first = _run(tg, kind, A, B, False, True)
+    for _ in range(3):
+        assert np.array_equal(_run(tg, kind, A, B, False, True), first)
 
 
 @pytest.mark.parametrize("kind", ["bf16", "f16"])

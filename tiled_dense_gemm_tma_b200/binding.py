@@ -20,7 +20,7 @@ STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
           6: "TG_ERR_NO_DEVICE"}
 
 # Every symbol include/tg_gemm.h declares.
-EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
+EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16", "tg_gemm_wfp4",
            "tg_gemm_f16_ex", "tg_gemm_bf16_ex", "tg_gemm_bf16_small_m_static",
            "tg_status_string", "tg_last_device_status", "tg_num_sms")
 
@@ -55,12 +55,13 @@ def load_library():
         lib.tg_gemm_f32.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, ci, vp]
         for name in ("tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_bf16_small_m_static"):
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci, vp]
-        lib.tg_gemm_w4a16.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
-                                      vp, i64, ci, vp]
+        for name in ("tg_gemm_w4a16", "tg_gemm_wfp4"):
+            getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
+                                           vp, i64, ci, vp]
         for name in ("tg_gemm_f16_ex", "tg_gemm_bf16_ex"):
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, ci, vp, i64, ci, vp, i64, ci, vp]
         for name in ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
-                     "tg_gemm_f16_ex", "tg_gemm_bf16_ex",
+                     "tg_gemm_wfp4", "tg_gemm_f16_ex", "tg_gemm_bf16_ex",
                      "tg_gemm_bf16_small_m_static", "tg_last_device_status"):
             getattr(lib, name).restype = ci
         lib.tg_status_string.argtypes = [ci]
@@ -288,6 +289,37 @@ def gemm_w4a16(A, Bq, scales, N, C=None, group_size=128, relu=False, stream=None
                                  group_size, C.data_ptr(), _ld(C, "C"),
                                  EPI_RELU if relu else EPI_NONE, _stream_handle(stream))
     _check(code, "tg_gemm_w4a16")
+    return C
+
+
+def gemm_wfp4(A, Bq, scales, N, C=None, block_size=32, relu=False, stream=None):
+    """C = epi(A @ W), W[k, n] = e2m1(code[k, n]) * 2^(scales[k // 32, n] - 127).
+
+    A: M x K bfloat16; Bq: K x ldbq uint8 (E2M1 codes, low nibble = even
+    column); scales: ceil(K / 32) x N uint8 E8M0 exponents; N: number of
+    output columns.  C is M x N bfloat16.
+    """
+    import torch
+    lib = load_library()
+    if A.dtype != torch.bfloat16 or Bq.dtype != torch.uint8 or scales.dtype != torch.uint8:
+        raise TypeError("A must be bfloat16, Bq and scales uint8")
+    if A.dim() != 2 or Bq.dim() != 2 or scales.dim() != 2:
+        raise ValueError("A, Bq and scales must be 2-D")
+    M, K = A.shape
+    if Bq.shape[0] != K:
+        raise ValueError("Bq must have K rows")
+    _require_cuda(A.device, (A, "A"), (Bq, "Bq"), (scales, "scales"))
+    if C is None:
+        C = empty_out(M, N, torch.bfloat16, A.device)
+    elif C.shape != (M, N) or C.dtype != torch.bfloat16:
+        raise ValueError("C has the wrong shape or dtype")
+    _require_cuda(A.device, (C, "C"))
+    with _device_ctx(A):
+        code = lib.tg_gemm_wfp4(M, N, K, A.data_ptr(), _ld(A, "A"), Bq.data_ptr(), _ld(Bq, "Bq"),
+                                scales.data_ptr(), _ld(scales, "scales"), block_size,
+                                C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
+                                _stream_handle(stream))
+    _check(code, "tg_gemm_wfp4")
     return C
 
 

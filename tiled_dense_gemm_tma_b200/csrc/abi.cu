@@ -87,6 +87,12 @@ tg::GemmArgs make_args(int64_t M, int64_t N, int64_t K, const void* A, int64_t l
 
 }  // namespace
 
+int tg::check_gemm_args(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                        const void* B, int64_t ldb, const void* C, int64_t ldc, int epilogue,
+                        int eb) {
+    return check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, eb);
+}
+
 extern "C" {
 
 tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K, const float* A, int64_t lda,
@@ -165,6 +171,32 @@ tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K, const void* A, int64_t 
     a.lds = lds;
     a.group = group_size;
     return static_cast<tg_status>(tg::launch_w4a16(a));
+}
+
+tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                       const uint8_t* Bq, int64_t ldbq, const uint8_t* scales, int64_t lds,
+                       int block_size, void* C, int64_t ldc, int epilogue, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
+    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if (block_size != 32) return TG_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return TG_OK;
+    if (!C || ldc < N) return TG_ERR_INVALID_ARG;
+    if (K > 0 && (!A || !Bq || !scales || lda < K || ldbq < (N + 1) / 2 || lds < N))
+        return TG_ERR_INVALID_ARG;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!pitch_ok(ldc, 2) ||
+        (K > 0 && (!pitch_ok(lda, 2) || !pitch_ok(ldbq, 1) || !pitch_ok(lds, 1))))
+        return TG_ERR_UNSUPPORTED;
+    if (!aligned16(C) || (ldc * 2) % 16 != 0) return TG_ERR_ALIGNMENT;
+    if (K > 0 && (!aligned16(A) || !aligned16(Bq) || !aligned16(scales) || (lda * 2) % 16 != 0 ||
+                  ldbq % 16 != 0 || lds % 16 != 0))
+        return TG_ERR_ALIGNMENT;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    tg::GemmArgs a = make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream);
+    a.scales = scales;
+    a.lds = lds;
+    a.group = block_size;
+    return static_cast<tg_status>(tg::launch_wfp4(a));
 }
 
 const char* tg_status_string(tg_status s) {

@@ -48,6 +48,7 @@ struct FfmaParams {
     float* ws;                // splits > 1: [tile][split][BM][BN] fp32 partials
     int* tickets;             // splits > 1: [tile], zero between calls
     int relu;
+    int inject;               // debug: 1 = CTA (0, 0, 0)'s producer skips arming the first slot
     unsigned long long timeout_ns;
     int* status;
     float* C;
@@ -129,6 +130,8 @@ ffma_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     ok = false;
                     break;
                 }
+                if (p.inject == 1 && kb == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+                    continue;                                   // debug: never arm slot 0
                 mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
                 armed |= 1u << s;
                 armed_par = (armed_par & ~(1u << s)) | (ph << s);
@@ -319,6 +322,7 @@ int launch_ffma_f32(const GemmArgs& a) {
     p.K = static_cast<int>(a.K);
     p.ldc = static_cast<int>(a.ldc);
     p.relu = a.relu;
+    p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = static_cast<float*>(a.C);

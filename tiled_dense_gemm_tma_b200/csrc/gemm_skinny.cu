@@ -1,6 +1,6 @@
-// gemm_skinny.cu -- launchers of the weight-streaming (small-M) kernel; its
-// split-K partials and tile tickets live in the per-stream workspace
-// (workspace.cu).
+// gemm_skinny.cu -- launchers of the weight-streaming (small-M) kernel, for
+// B stored K x N (the plain call) or N x K (a transposed-B call); its split-K
+// partials and tile tickets live in the per-stream workspace (workspace.cu).
 #include "gemm_skinny.cuh"
 #include "host.cuh"
 #include "launch.h"
@@ -9,9 +9,9 @@ namespace tg {
 
 namespace {
 
-template <WKind W, int MPAD>
+template <WKind W, int MPAD, int WK>
 int run(const GemmArgs& a) {
-    using Cfg = SkCfg<W, MPAD>;
+    using Cfg = SkCfg<W, MPAD, WK>;
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
@@ -28,9 +28,23 @@ int run(const GemmArgs& a) {
         if (!tensor_map_2d(&tW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
                            Cfg::GN / 2, Cfg::BK, SWZ_128))
             return kCudaError;
-        if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
-                           a.lds * 2, Cfg::GN, 1, SWZ_NONE))
+        if constexpr (Cfg::FP4) {
+            // E8M0 bytes: ceil(K / 32) rows of N; two rows (64 k) per unit
+            if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, (a.K + 31) / 32,
+                               a.lds, Cfg::GN, Cfg::BK / 32, SWZ_NONE))
+                return kCudaError;
+        } else {
+            if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
+                               a.lds * 2, Cfg::GN, 1, SWZ_NONE))
+                return kCudaError;
+        }
+    } else if constexpr (WK) {
+        // B stored N x K: boxes of 64 k x the tile's 128 stored rows
+        const CUtensorMapDataType dt = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        if (!tensor_map_2d(&tW, a.B, dt, 2, a.K, a.N, a.ldb * 2, 64, Cfg::TN, SWZ_128))
             return kCudaError;
+        tS = tW;                                   // unused
     } else {
         const CUtensorMapDataType dt = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -38,13 +52,15 @@ int run(const GemmArgs& a) {
             return kCudaError;
         tS = tW;                                   // unused
     }
-    const CUtensorMapDataType xt = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType xt = Cfg::OUTW == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!tensor_map_2d(&tX, a.A, xt, 2, a.K, a.M, a.lda * 2, 64, MPAD, SWZ_128))
         return kCudaError;
 
     auto kern = skinny_kernel<Cfg>;
-    const int slot = 16 + static_cast<int>(W) * 4 + (MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3);
+    const int mi = MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3;
+    const int slot = W == WKind::FP4 ? 36 + mi
+                   : WK ? 28 + static_cast<int>(W) * 4 + mi : 16 + static_cast<int>(W) * 4 + mi;
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
         return kCudaError;
     SkParams p;
@@ -56,6 +72,7 @@ int run(const GemmArgs& a) {
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;
@@ -68,12 +85,12 @@ int run(const GemmArgs& a) {
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
 }
 
-template <WKind W>
+template <WKind W, int WK = 0>
 int dispatch(const GemmArgs& a) {
-    if (a.M <= 16) return run<W, 16>(a);
-    if (a.M <= 32) return run<W, 32>(a);
-    if (a.M <= 64) return run<W, 64>(a);
-    return run<W, 128>(a);
+    if (a.M <= 16) return run<W, 16, WK>(a);
+    if (a.M <= 32) return run<W, 32, WK>(a);
+    if (a.M <= 64) return run<W, 64, WK>(a);
+    return run<W, 128, WK>(a);
 }
 
 }  // namespace
@@ -81,5 +98,9 @@ int dispatch(const GemmArgs& a) {
 int launch_skinny_bf16(const GemmArgs& a) { return dispatch<WKind::BF16>(a); }
 int launch_skinny_f16(const GemmArgs& a) { return dispatch<WKind::F16>(a); }
 int launch_skinny_w4a16(const GemmArgs& a) { return dispatch<WKind::INT4>(a); }
+int launch_skinny_wfp4(const GemmArgs& a) { return dispatch<WKind::FP4>(a); }
+int launch_skinny_trans_b(const GemmArgs& a, int bf16) {
+    return bf16 ? dispatch<WKind::BF16, 1>(a) : dispatch<WKind::F16, 1>(a);
+}
 
 }  // namespace tg

@@ -9,7 +9,8 @@
 //   D[n][m] = sum_k W[k][n] * X[m][k]        (C = D^T, X = A)
 //
 // * The weight tile (128 columns n x BK rows k) is the MMA's 128-row operand,
-//   N-major in shared memory; the activations (MPAD >= M rows, zero-padded
+//   N-major in shared memory (K-major when B is stored transposed, N x K, as
+//   in the backward product dA = dC . B^T); the activations (MPAD >= M rows, zero-padded
 //   by the copy engine) are the MMA's N operand, K-major.  D lives in TMEM as
 //   128 lanes (n) x MPAD columns (m).
 // * Stream-K: the (column group, k-unit) units of all T = ceil(N/GN) column
@@ -23,7 +24,9 @@
 //   in segment order -- deterministic -- applies ReLU, rounds and writes C,
 //   and resets the ticket for the next call.
 // * Weights arrive either as fp16/bf16 tiles by TMA, or as packed 4-bit
-//   weights + scales that converter warps expand (dequant.cuh).
+//   weights + scales that converter warps expand (dequant.cuh): signed
+//   integers with fp16 group scales into fp16 tiles, or FP4 (E2M1) codes
+//   with E8M0 block scales into bf16 tiles.
 #pragma once
 #include "ptx.cuh"
 #include "dequant.cuh"
@@ -33,14 +36,25 @@
 
 namespace tg {
 
-enum class WKind { F16 = 0, BF16 = 1, INT4 = 2 };
+// Weight kinds: 16-bit weights, signed 4-bit integers with fp16 group scales
+// (fp16 activations and output), FP4 E2M1 codes with E8M0 block scales
+// (bf16 activations and output).
+enum class WKind { F16 = 0, BF16 = 1, INT4 = 2, FP4 = 3 };
 
-template <WKind W_, int MPAD_>
+// WK_ = 1: 16-bit weights stored transposed (B is N x K row-major, the
+// op(B) = B^T of a transposed-operand call): each weight tile arrives as
+// BK/64 boxes of 128 stored rows (the tile's n) x 64 k and the MMA reads it
+// K-major.  WK_ = 0: B is K x N row-major, tiles arrive N-major.
+template <WKind W_, int MPAD_, int WK_ = 0>
 struct SkCfg {
     static constexpr WKind W = W_;
     static constexpr int MPAD = MPAD_;                  // MMA N: 16, 32, 64 or 128
+    static constexpr int WK = WK_;
     static constexpr int TN = 128;                      // weight columns per MMA (MMA M)
-    static constexpr bool Q4 = W_ == WKind::INT4;
+    static constexpr bool Q4 = W_ == WKind::INT4 || W_ == WKind::FP4;   // packed 4-bit weights
+    static constexpr bool FP4 = W_ == WKind::FP4;
+    // activation, MMA operand and output type
+    static constexpr WKind OUTW = (W_ == WKind::BF16 || W_ == WKind::FP4) ? WKind::BF16 : WKind::F16;
     // k rows per unit: 16-bit weights come in 128-row boxes (taller TMA
     // copies stream faster), 4-bit weights in 64-row slices
     static constexpr int BK = Q4 ? 64 : 128;
@@ -54,7 +68,9 @@ struct SkCfg {
     static constexpr int X_SLICE = MPAD * 128;          // MPAD rows x 64 fp16
     static constexpr int X_BYTES = KSL * X_SLICE;
     static constexpr int Q_BYTES = Q4 ? BK * GN / 2 : 0;   // 8 KB packed
-    static constexpr int S_BYTES = Q4 ? GN * 2 : 0;        // 512 B scales
+    // 512 B of scales per unit: one row of GN fp16 group scales (a 128-row
+    // group) or two rows of GN E8M0 bytes (two 32-row blocks)
+    static constexpr int S_BYTES = Q4 ? GN * 2 : 0;
     // Ring of TMA-filled slots.  16-bit weights: [W | X], released by the MMA.
     // 4-bit weights: [Q | S], released by the converters as soon as they have
     // expanded it into a second ring of fp16 tiles; the activations then
@@ -95,6 +111,8 @@ struct SkCfg {
     static_assert(RAW_STAGES >= 3, "ring");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
     static_assert(!Q4 || GN / 2 == 128, "packed row");
+    static_assert(!WK || (!Q4 && W_CHUNK == 64 * 2 * BK && TN * 128 == 16384),
+                  "K-major weights: 16-bit only; BK/64 boxes of 128 rows x 128 B fill W_BYTES");
 };
 
 struct SkParams {
@@ -102,6 +120,7 @@ struct SkParams {
     int relu;
     int T, KB, U;             // column groups (GN wide), k-slices per group, units = T * KB
     int J;                    // workspace slots per tile (max segments of a tile)
+    int inject;               // debug: 1 = CTA 0's producer skips arming the first slot
     unsigned long long timeout_ns;
     int* status;
     void* C;
@@ -237,14 +256,28 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     const int xs = it % Cfg::X_STAGES;
                     const uint32_t xph = (it / Cfg::X_STAGES) & 1;
                     if (!bounded_wait(&xempty[xs], xph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                    if (p.inject == 1 && it == 0 && c == 0) continue;   // debug: never arm slot 0
                     mbar_arrive_expect_tx(&full[s], Cfg::Q_BYTES + Cfg::S_BYTES);
                     tma_load_2d(slot_q(s), &tmW, &full[s], t * (Cfg::GN / 2), kb * Cfg::BK);
-                    tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::GN, (kb * Cfg::BK) / 128);
+                    tma_load_2d(slot_s(s), &tmS, &full[s], t * Cfg::GN,
+                                (kb * Cfg::BK) / (Cfg::FP4 ? 32 : 128));
                     mbar_arrive_expect_tx(&xfull[xs], Cfg::X_BYTES);
                     tma_load_2d(xring + xs * Cfg::X_BYTES, &tmX, &xfull[xs], kb * Cfg::BK, 0);
                     xarmed |= 1u << xs;
                     xarmed_par = (xarmed_par & ~(1u << xs)) | (xph << xs);
+                } else if constexpr (Cfg::WK) {
+                    if (p.inject == 1 && it == 0 && c == 0) continue;   // debug: never arm slot 0
+                    // B stored N x K: BK/64 boxes of the tile's 128 n rows x 64 k
+                    // (rows past N read the copy engine's zero fill)
+                    mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + Cfg::W_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < Cfg::KSL; ++ks) {
+                        tma_load_2d(slot_w(s) + ks * (Cfg::TN * 128), &tmW, &full[s],
+                                    kb * Cfg::BK + 64 * ks, t * Cfg::TN);
+                        tma_load_2d(slot_x(s) + ks * Cfg::X_SLICE, &tmX, &full[s], kb * Cfg::BK + 64 * ks, 0);
+                    }
                 } else {
+                    if (p.inject == 1 && it == 0 && c == 0) continue;   // debug: never arm slot 0
                     // the second 64-column box is skipped when it starts past N
                     const bool second = t * Cfg::TN + 64 < p.N;
                     mbar_arrive_expect_tx(&full[s], Cfg::X_BYTES + (second ? 2 : 1) * Cfg::W_CHUNK);
@@ -276,8 +309,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (elect_one()) {
-            constexpr uint32_t fmt = Cfg::W == WKind::BF16 ? 1u : 0u;
-            constexpr uint32_t idesc = make_idesc(fmt, Cfg::TN, Cfg::MPAD, 1, 0);
+            constexpr uint32_t fmt = Cfg::OUTW == WKind::BF16 ? 1u : 0u;
+            constexpr uint32_t idesc = make_idesc(fmt, Cfg::TN, Cfg::MPAD, Cfg::WK ? 0 : 1, 0);
             bool ok = true;
             int it = 0, seg = 0;
             uint32_t d_tmem = tmem_base;
@@ -318,9 +351,12 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 for (int j = 0; j < Cfg::NSUB; ++j) {
 #pragma unroll
                     for (int k = 0; k < Cfg::BK / 16; ++k) {
-                        // weights: N-major, 16 k rows of 128 B per MMA; activations: K-major
-                        const uint64_t ad = sw128_desc(w_addr + j * 2 * Cfg::W_CHUNK + k * 16 * 128,
-                                                       Cfg::W_CHUNK, 1024);
+                        // weights: N-major, 16 k rows of 128 B per MMA (or, stored
+                        // transposed, K-major: 32 B of k inside the 128-byte rows of
+                        // the k/4-th box); activations: K-major
+                        const uint64_t ad = Cfg::WK
+                            ? sw128_desc(w_addr + (k >> 2) * (Cfg::TN * 128) + (k & 3) * 32, 16, 1024)
+                            : sw128_desc(w_addr + j * 2 * Cfg::W_CHUNK + k * 16 * 128, Cfg::W_CHUNK, 1024);
                         const uint64_t bd = sw128_desc(x_addr + (k >> 2) * Cfg::X_SLICE + (k & 3) * 32,
                                                        16, 1024);
                         const int set = k % Cfg::R;
@@ -398,7 +434,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                             const int m = mc + i;
                             if (m >= p.M) break;
                             const float x = __uint_as_float(v[i]);
-                            if (n < p.N) store_out<Cfg::W>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
+                            if (n < p.N) store_out<Cfg::OUTW>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
                         }
                     } else {
                         float* col = slot + nj;
@@ -484,7 +520,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                             if (p.relu)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) o[e] = fmaxf(o[e], 0.f);
-                            store_out4<Cfg::W>(p.C, p.ldc, m, n, p.N, o);
+                            store_out4<Cfg::OUTW>(p.C, p.ldc, m, n, p.N, o);
                         }
                     }
                 }
@@ -503,8 +539,12 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status) ||
                     !bounded_wait(&wempty[w], wph ^ 1, abort_flag, limit, p.status))
                     break;
-                dequant_slice<Cfg::BK, Cfg::GN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
-                    slot_q(s), slot_s(s), wring + w * Cfg::W_BYTES, ctid);
+                if constexpr (Cfg::FP4)
+                    dequant_slice_fp4<Cfg::BK, Cfg::GN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
+                        slot_q(s), slot_s(s), wring + w * Cfg::W_BYTES, ctid);
+                else
+                    dequant_slice<Cfg::BK, Cfg::GN, 32 * Cfg::CONV_WARPS, Cfg::W_CHUNK>(
+                        slot_q(s), slot_s(s), wring + w * Cfg::W_BYTES, ctid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {

@@ -125,6 +125,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.inject = 0;
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = C;
@@ -143,15 +144,12 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
 extern "C" tg_status tg_gemm_bf16_small_m_static(int64_t M, int64_t N, int64_t K, const void* A,
                                                  int64_t lda, const void* B, int64_t ldb, void* C,
                                                  int64_t ldc, int epilogue, void* stream) {
-    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
-    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return TG_OK;
+    // the checks of every other entry point (sizes, pointers, leading
+    // dimensions, row-pitch bound, alignment), before any CUDA call
+    const tg_status s = static_cast<tg_status>(
+        tg::check_gemm_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2));
+    if (s != TG_OK || M == 0 || N == 0) return s;
     if (M > 128) return TG_ERR_UNSUPPORTED;            // the small-M kernel's limit
-    if (!C || ldc < N || (K > 0 && (!A || !B || lda < K || ldb < N))) return TG_ERR_INVALID_ARG;
-    if (N > 0x7fffffffll || K > 0x7fffffffll) return TG_ERR_UNSUPPORTED;
-    auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (!al(C) || (ldc * 2) % 16) return TG_ERR_ALIGNMENT;
-    if (K > 0 && (!al(A) || !al(B) || (lda * 2) % 16 || (ldb * 2) % 16)) return TG_ERR_ALIGNMENT;
     int dev = 0;
     const tg::DeviceInfo* di = tg::current_device(&dev);
     if (!di || dev >= tg::kMaxDevs) return TG_ERR_NO_DEVICE;

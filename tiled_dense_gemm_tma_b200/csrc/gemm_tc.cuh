@@ -74,7 +74,7 @@ struct TcCfg {
 struct TcParams {
     int M, N, K;
     int relu;
-    int inject;               // debug: 1 = producer skips arming the first slot
+    int inject;               // debug: 1 = CTA 0's producer skips arming the first slot
     unsigned long long timeout_ns;
     int* status;              // device status word (ST_TIMEOUT on an expired wait)
     void* C;                  // output base and row pitch (elements), for the ragged
@@ -261,7 +261,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
-                    if (p.inject == 1 && it == 0) continue;   // debug: never arm slot 0
+                    if (p.inject == 1 && it == 0 && blockIdx.x == 0) continue;   // debug: never arm slot 0
                     // B boxes that start past column N are not loaded: their
                     // columns only feed output columns >= N, which are never stored.
                     const int live_chunks = min(Cfg::BN / Cfg::CHUNK_N,

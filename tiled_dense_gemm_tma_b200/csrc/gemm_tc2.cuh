@@ -132,7 +132,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
-                    if (p.inject == 1 && it == 0 && rank == 0) continue;   // debug: never arm slot 0
+                    if (p.inject == 1 && it == 0 && pair == 0 && rank == 0) continue;   // debug: never arm slot 0
                     const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
                     mbar_arrive_expect_tx_cluster(fbar, bytes);
                     armed |= 1u << s;

@@ -1,7 +1,10 @@
 // gemm_w4a16.cu -- dequantize GEMM C = epi(A . W) with fp16 activations A
 // (M x K, row-major) and 4-bit weights W = fp16(q * s) (see dequant.cuh),
-// fp32 accumulation in tensor memory, fp16 output.  This launcher serves the
-// large-M case; small M goes to the weight-streaming kernel (gemm_skinny.cu).
+// fp32 accumulation in tensor memory, fp16 output; and the same kernel for
+// FP4 weights (E2M1 codes with E8M0 block scales, bf16 activations, W formed
+// exactly in bf16, bf16 output).  One CTA per 128 x 256 tile: the large-M
+// path when a CTA-pair launch is refused (gemm_w4a16_pair.cu is the default);
+// small M goes to the weight-streaming kernel (gemm_skinny.cu).
 //
 // The unpack and group scale are fused into operand staging:
 //   warp 0      TMA producer: per K slice (BK = 64) loads the A box (BM x 64
@@ -56,6 +59,10 @@ struct W4 {
     static_assert(TMEM_COLS == 512, "TMEM: two 256-column accumulators");
 };
 
+// QFP4 = false: signed 4-bit weights with fp16 group scales, fp16
+// activations and output; true: FP4 (E2M1) weights with E8M0 block scales,
+// bf16 activations and output (dequant.cuh).
+template <bool QFP4>
 __global__ void __launch_bounds__(W4::THREADS, 1)
 w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                   const __grid_constant__ CUtensorMap tmQ,
@@ -86,7 +93,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int ntm = (p.M + W4::BM - 1) / W4::BM;
     const int ntn = (p.N + W4::BN - 1) / W4::BN;
     const int num_tiles = ntm * ntn;
-    const int num_kb = p.K / W4::BK;                     // K is a multiple of 128
+    const int num_kb = (p.K + W4::BK - 1) / W4::BK;      // past K: zero-filled codes and activations
     const uint64_t limit = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -129,13 +136,14 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t s = it % W4::RAW_STAGES;
                     const uint32_t ph = (it / W4::RAW_STAGES) & 1;
                     if (!bounded_wait(&rempty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                    if (p.inject == 1 && it == 0 && blockIdx.x == 0) continue;   // debug: never arm slot 0
                     mbar_arrive_expect_tx(&full[s], W4::A_BYTES + W4::Q_BYTES + W4::S_BYTES);
                     armed |= 1u << s;
                     armed_par = (armed_par & ~(1u << s)) | (ph << s);
                     tma_load_2d(smA + s * W4::A_BYTES, &tmA, &full[s], kb * W4::BK, tm * W4::BM);
                     tma_load_2d(smQ + s * W4::Q_BYTES, &tmQ, &full[s], tn * (W4::BN / 2), kb * W4::BK);
                     tma_load_2d(smS + s * W4::S_BYTES, &tmS, &full[s], tn * W4::BN,
-                                (kb * W4::BK) / 128);
+                                (kb * W4::BK) / (QFP4 ? 32 : 128));
                 }
             }
             if (!ok) {
@@ -150,7 +158,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (elect_one()) {
-            constexpr uint32_t idesc = make_idesc(0, W4::BM, W4::BN, 0, 1);
+            constexpr uint32_t idesc = make_idesc(QFP4 ? 1 : 0, W4::BM, W4::BN, 0, 1);
             uint32_t it = 0, tl = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tl) {
@@ -198,7 +206,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
             tc_fence_after();
-            epilogue_tile<OutT::F16, W4::BN, true, 1>(&tmC, p, tmem_base + acc * W4::BN, q, lane,
+            epilogue_tile<QFP4 ? OutT::BF16 : OutT::F16, W4::BN, true, 1>(&tmC, p, tmem_base + acc * W4::BN, q, lane,
                                                       tm * W4::BM + q * 32, tn * W4::BN, stg0,
                                                       nstore);
             tc_fence_before();
@@ -220,8 +228,12 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t bph = (it / W4::B_STAGES) & 1;
                 if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status) ||
                     !bounded_wait(&bempty[b], bph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
-                dequant_slice<W4::BK, W4::BN, 32 * W4::CONV_WARPS, W4::B_CHUNK>(
-                    smQ + s * W4::Q_BYTES, smS + s * W4::S_BYTES, smB + b * W4::B_BYTES, ctid);
+                if constexpr (QFP4)
+                    dequant_slice_fp4<W4::BK, W4::BN, 32 * W4::CONV_WARPS, W4::B_CHUNK>(
+                        smQ + s * W4::Q_BYTES, smS + s * W4::S_BYTES, smB + b * W4::B_BYTES, ctid);
+                else
+                    dequant_slice<W4::BK, W4::BN, 32 * W4::CONV_WARPS, W4::B_CHUNK>(
+                        smQ + s * W4::Q_BYTES, smS + s * W4::S_BYTES, smB + b * W4::B_BYTES, ctid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -240,26 +252,27 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
 }
 
-}  // namespace
-
-int launch_w4a16_large(const GemmArgs& a) {
+template <bool QFP4>
+int run_large(const GemmArgs& a) {
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
+    const CUtensorMapDataType at = QFP4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tA, tQ, tS, tC;
-    if (!tensor_map_2d(&tA, a.A, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.K, a.M, a.lda * 2,
-                       W4::BK, W4::BM, SWZ_128))
+    if (!tensor_map_2d(&tA, a.A, at, 2, a.K, a.M, a.lda * 2, W4::BK, W4::BM, SWZ_128))
         return kCudaError;
     if (!tensor_map_2d(&tQ, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
                        W4::BN / 2, W4::BK, SWZ_128))
         return kCudaError;
-    if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
-                       a.lds * 2, W4::BN, 1, SWZ_NONE))
+    if (QFP4 ? !tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, (a.K + 31) / 32,
+                              a.lds, W4::BN, W4::BK / 32, SWZ_NONE)
+             : !tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
+                              a.lds * 2, W4::BN, 1, SWZ_NONE))
         return kCudaError;
-    if (!tensor_map_2d(&tC, a.C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.M, a.ldc * 2,
-                       64, 32, SWZ_128))
+    if (!tensor_map_2d(&tC, a.C, at, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
         return kCudaError;
-    if (set_smem_attr(reinterpret_cast<const void*>(w4a16_gemm_kernel), W4::SMEM_BYTES, 9) !=
+    auto kern = w4a16_gemm_kernel<QFP4>;
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), W4::SMEM_BYTES, QFP4 ? 6 : 9) !=
         cudaSuccess)
         return kCudaError;
     const long long tiles = ((a.M + W4::BM - 1) / W4::BM) * ((a.N + W4::BN - 1) / W4::BN);
@@ -269,15 +282,20 @@ int launch_w4a16_large(const GemmArgs& a) {
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
-    p.inject = 0;
+    p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;
     p.ldc = a.ldc;
     if (!p.status) return kCudaError;
-    w4a16_gemm_kernel<<<grid, W4::THREADS, W4::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(
+    kern<<<grid, W4::THREADS, W4::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(
         tA, tQ, tS, tC, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
 }
+
+}  // namespace
+
+int launch_w4a16_large(const GemmArgs& a) { return run_large<false>(a); }
+int launch_wfp4_large(const GemmArgs& a) { return run_large<true>(a); }
 
 }  // namespace tg

@@ -1,6 +1,8 @@
 // gemm_w4a16_pair.cu -- the dequantize GEMM (fp16 activations x signed 4-bit
 // weights with fp16 group scales, "W4A16" of the pages' dequantize-GEMM
-// examples) for M > 128, on CTA pairs (tcgen05 cta_group::2).
+// examples) for M > 128, on CTA pairs (tcgen05 cta_group::2); the same kernel
+// serves FP4 weights (E2M1 codes with E8M0 block scales, bf16 activations,
+// bf16 operand and output: the WFP4 GEMM).
 //
 // The one-CTA kernel (gemm_w4a16.cu) is bound by shared-memory bandwidth:
 // per 128 x 256 x 64 step its MMAs read 48 KB of operands and its converter
@@ -98,6 +100,10 @@ __device__ __forceinline__ bool bounded_wait_cluster(uint64_t* bar, uint32_t par
 }
 
 
+// QFP4 = false: signed 4-bit weights with fp16 group scales, fp16
+// activations and output; true: FP4 (E2M1) weights with E8M0 block scales,
+// bf16 activations and output (dequant.cuh).
+template <bool QFP4>
 __global__ void __launch_bounds__(W4P::THREADS, 1)
 w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                   const __grid_constant__ CUtensorMap tmQ,
@@ -187,6 +193,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t ph = (it / W4P::STAGES) & 1;
                     if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status) ||
                         !bounded_wait(&rempty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                    if (p.inject == 1 && it == 0 && pair == 0 && rank == 0) continue;   // debug: never arm slot 0
                     const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
                     mbar_arrive_expect_tx_cluster(fbar, a_live ? W4P::A_STAGE : 0);
                     armed |= 1u << s;
@@ -196,7 +203,8 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                     rarmed |= 1u << s;
                     rarmed_par = (rarmed_par & ~(1u << s)) | (ph << s);
                     tma_load_2d(smQ + s * W4P::Q_BYTES, &tmQ, &rfull[s], n0 / 2, kb * W4P::BK);
-                    tma_load_2d(smS + s * W4P::S_BYTES, &tmS, &rfull[s], n0, (kb * W4P::BK) / 128);
+                    tma_load_2d(smS + s * W4P::S_BYTES, &tmS, &rfull[s], n0,
+                                (kb * W4P::BK) / (QFP4 ? 32 : 128));
                 }
             }
             if (!ok) {
@@ -219,7 +227,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     } else if (warp == 1) {
         // ------------------------------------------ MMA issuer (leader only)
         if (rank == 0 && elect_one()) {
-            constexpr uint32_t idesc = make_idesc(0, W4P::PM, W4P::BN, 0, 1);
+            constexpr uint32_t idesc = make_idesc(QFP4 ? 1 : 0, W4P::PM, W4P::BN, 0, 1);
             uint32_t it = 0, tl = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs, ++tl) {
@@ -273,7 +281,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
             tc_fence_after();
-            epilogue_tile<OutT::F16, W4P::BN, true, 2>(&tmC, p, tmem_base + acc * W4P::BN, q, lane,
+            epilogue_tile<QFP4 ? OutT::BF16 : OutT::F16, W4P::BN, true, 2>(&tmC, p, tmem_base + acc * W4P::BN, q, lane,
                                                        tm * W4P::PM + rank * W4P::BM + q * 32,
                                                        tn * W4P::BN, stg0, nstore);
             tc_fence_before();
@@ -295,8 +303,12 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t bph = (it / W4P::B_STAGES) & 1;
                 if (!bounded_wait(&rfull[s], ph, abort_flag, limit, p.status) ||
                     !bounded_wait(&bempty[b], bph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
-                dequant_slice<W4P::BK, W4P::HN, 32 * W4P::CONV_WARPS, W4P::B_CHUNK>(
-                    smQ + s * W4P::Q_BYTES, smS + s * W4P::S_BYTES, smB + b * W4P::B_STAGE, ctid);
+                if constexpr (QFP4)
+                    dequant_slice_fp4<W4P::BK, W4P::HN, 32 * W4P::CONV_WARPS, W4P::B_CHUNK>(
+                        smQ + s * W4P::Q_BYTES, smS + s * W4P::S_BYTES, smB + b * W4P::B_STAGE, ctid);
+                else
+                    dequant_slice<W4P::BK, W4P::HN, 32 * W4P::CONV_WARPS, W4P::B_CHUNK>(
+                        smQ + s * W4P::Q_BYTES, smS + s * W4P::S_BYTES, smB + b * W4P::B_STAGE, ctid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -316,29 +328,30 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     }
 }
 
-}  // namespace
-
 // Returns kUnsupported (nothing launched) when the pair launch is refused,
 // so the caller can fall back to the one-CTA kernel.
-int launch_w4a16_pair(const GemmArgs& a) {
+template <bool QFP4>
+int run_pair(const GemmArgs& a) {
     if (pair_kernels_disabled()) return kUnsupported;
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
+    const CUtensorMapDataType at = QFP4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tA, tQ, tS, tC;
-    if (!tensor_map_2d(&tA, a.A, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.K, a.M, a.lda * 2,
-                       W4P::BK, W4P::BM, SWZ_128))
+    if (!tensor_map_2d(&tA, a.A, at, 2, a.K, a.M, a.lda * 2, W4P::BK, W4P::BM, SWZ_128))
         return kCudaError;
     if (!tensor_map_2d(&tQ, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
                        W4P::HN / 2, W4P::BK, SWZ_64))
         return kCudaError;
-    if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
-                       a.lds * 2, W4P::HN, 1, SWZ_NONE))
+    if (QFP4 ? !tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, (a.K + 31) / 32,
+                              a.lds, W4P::HN, W4P::BK / 32, SWZ_NONE)
+             : !tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
+                              a.lds * 2, W4P::HN, 1, SWZ_NONE))
         return kCudaError;
-    if (!tensor_map_2d(&tC, a.C, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.M, a.ldc * 2,
-                       64, 32, SWZ_128))
+    if (!tensor_map_2d(&tC, a.C, at, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
         return kCudaError;
-    if (set_smem_attr(reinterpret_cast<const void*>(w4a16_pair_kernel), W4P::SMEM_BYTES, 10) !=
+    auto kern = w4a16_pair_kernel<QFP4>;
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), W4P::SMEM_BYTES, QFP4 ? 7 : 10) !=
         cudaSuccess)
         return kCudaError;
     const long long tiles = ((a.M + W4P::PM - 1) / W4P::PM) * ((a.N + W4P::BN - 1) / W4P::BN);
@@ -349,7 +362,7 @@ int launch_w4a16_pair(const GemmArgs& a) {
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
-    p.inject = 0;
+    p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;
@@ -367,11 +380,16 @@ int launch_w4a16_pair(const GemmArgs& a) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, w4a16_pair_kernel, tA, tQ, tS, tC, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tQ, tS, tC, p) != cudaSuccess) {
         cudaGetLastError();                       // clear; caller falls back
         return kUnsupported;
     }
     return kOk;
 }
+
+}  // namespace
+
+int launch_w4a16_pair(const GemmArgs& a) { return run_pair<false>(a); }
+int launch_wfp4_pair(const GemmArgs& a) { return run_pair<true>(a); }
 
 }  // namespace tg

@@ -172,6 +172,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 const int s = it % Cfg::STAGES;
                 const uint32_t ph = (it / Cfg::STAGES) & 1;
                 if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
+                if (p.inject == 1 && it == 0 && c == 0) continue;   // debug: never arm slot 0
                 uint8_t* slot = ring + s * Cfg::SLOT;
                 uint8_t* xs = slot + Cfg::W_BYTES + Cfg::S_BYTES;
                 if constexpr (Cfg::Q4) {
@@ -437,6 +438,7 @@ int run_gemv(const GemmArgs& a) {
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;

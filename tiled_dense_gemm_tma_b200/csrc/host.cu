@@ -130,7 +130,9 @@ int inject_mode() {
         const char* e = std::getenv("TG_INJECT");
         return e ? std::atoi(e) : 0;
     }();
-    return v;
+    static std::atomic<int> taken{0};
+    if (v == 0) return 0;
+    return taken.exchange(1) == 0 ? v : 0;      // the first launch only
 }
 
 bool pair_kernels_disabled() {

@@ -31,7 +31,13 @@ constexpr CUtensorMapSwizzle SWZ_128_32B = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
 // Bounded-wait limit for kernels, in ns (TG_DEBUG_TIMEOUT_US overrides).
 unsigned long long wait_limit_ns();
 
-// Debug fault-injection selector (TG_INJECT, default 0 = off).
+// Debug fault injection (TG_INJECT, default 0 = off), read once per process.
+// With TG_INJECT=1 the first kernel launch of the process (and only that
+// one) has the TMA producer of CTA 0 (of CTA pair 0's leader) skip arming its
+// first ring slot: that CTA's consumers wait on a barrier nothing completes,
+// run into the bounded-wait limit, report TG_ERR_TIMEOUT and return, while
+// the other CTAs finish (leaving split-K tickets incomplete).  Launchers
+// call this once per launch.
 int inject_mode();
 // Debug: TG_NO_PAIR=1 makes every CTA-pair launch report "unsupported", so
 // the calls take the one-CTA kernels (the path used when a cluster launch is
@@ -47,7 +53,9 @@ int* device_status_ptr();
 //    0-4   gemm_tc.cu        one-CTA bf16/f16/tf32, CTA-pair bf16/f16
 //    5, 11-15 gemm_tc.cu     CTA-pair with transposed operands
 //    8     gemm_ffma.cu      9  gemm_w4a16.cu     10  gemm_w4a16_pair.cu
-//   16-27  gemm_skinny.cu    40-48  gemv.cu       50-53  gemm_skinny_static.cu
+//   16-27  gemm_skinny.cu    28-35  gemm_skinny.cu (weights stored transposed)
+//   36-39  gemm_skinny.cu (FP4 weights)
+//   40-48  gemv.cu           50-53  gemm_skinny_static.cu
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 
 }  // namespace tg

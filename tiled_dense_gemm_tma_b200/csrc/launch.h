@@ -14,8 +14,8 @@ struct GemmArgs {
     const void* A; int64_t lda;      // elements
     const void* B; int64_t ldb;      // elements (bytes for packed 4-bit weights)
     void* C; int64_t ldc;            // elements
-    const void* scales; int64_t lds; // 4-bit path only
-    int group;                       // 4-bit path only
+    const void* scales; int64_t lds; // 4-bit paths only (lds: elements, bytes for E8M0 scales)
+    int group;                       // 4-bit paths only
     int relu;
     void* stream;
 };
@@ -28,13 +28,26 @@ int launch_ffma_f32(const GemmArgs& a);
 int launch_w4a16(const GemmArgs& a);
 int launch_w4a16_large(const GemmArgs& a);
 int launch_w4a16_pair(const GemmArgs& a);
+// FP4 (E2M1 + E8M0) weights, bf16 activations: scales / lds in bytes.
+int launch_wfp4(const GemmArgs& a);
+int launch_wfp4_large(const GemmArgs& a);
+int launch_wfp4_pair(const GemmArgs& a);
+int launch_skinny_wfp4(const GemmArgs& a);
 int launch_skinny_bf16(const GemmArgs& a);
 int launch_skinny_f16(const GemmArgs& a);
 int launch_skinny_w4a16(const GemmArgs& a);
+// 16-bit weights stored transposed (B is N x K): the weight-streaming kernel
+// reading K-major weight tiles.
+int launch_skinny_trans_b(const GemmArgs& a, int bf16);
 int launch_gemv_bf16(const GemmArgs& a);
 int launch_gemv_f16(const GemmArgs& a);
 int launch_gemv_w4a16(const GemmArgs& a);
 void mark_workspaces_dirty(int dev);
+// The argument checks every 16-bit and fp32 entry point runs before any CUDA
+// call (sizes, pointers, leading dimensions, the row-pitch bound, alignment)
+// for elements of `eb` bytes; returns a tg_status value.
+int check_gemm_args(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, const void* B,
+                    int64_t ldb, const void* C, int64_t ldc, int epilogue, int eb);
 // Per-(device, stream) scratch of the split-K paths: `tickets` ints (zero
 // between calls) and `partial_bytes` of fp32 partials.
 bool stream_workspace(int dev, void* stream, long long tickets, long long partial_bytes,
