@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference] [--no-breakdown]
+    python bench.py --sweep        (one GPU: rewrite the built-in tuning rules)
 
 A step is one call of the whole hot path for one GEMM of the workload:
 argument validation and tensor-map lookup on the host, then the persistent
@@ -478,6 +479,132 @@ def oracle_rate(name, host, budget_s):
     return flops / t, desc, oracle.num_threads(), t
 
 
+# ------------------------------------------------------------ offline sweep
+#
+# Shape classes of the tuning table: (op, m_lo, m_hi, n_lo, n_hi), the
+# configured workloads that represent the class, and the candidate launch
+# shapes timed for it.  The all-default candidate is always timed first; a
+# class gets a built-in rule only when another candidate beats it by more
+# than SWEEP_MARGIN on the geometric mean of its workloads' times.
+INF = (1 << 63) - 1
+_PAIR16 = ([{"path": "cta_pair", "stages": st, "group_m": g} for st in (4, 6) for g in (4, 8, 16)] +
+           [{"path": "one_cta", "group_m": g} for g in (8, 16)])
+_SMALL = [{"path": "small_m", "ctas": c} for c in (140, 128, 112, 96, 74)]
+SWEEP_CLASSES = [
+    ("bf16", 5, 64, 1, INF, ["bf16_gemm_16x8192x8192"], _SMALL + [{"path": "cta_pair"}]),
+    ("bf16", 65, 128, 1, INF, ["bf16_gemm_128x14336x4096"], _SMALL + [{"path": "cta_pair"}]),
+    ("bf16", 129, INF, 1, INF, ["bf16_gemm_8192", "bf16_gemm_4096", "bf16_gemm_8192x1024x8192",
+                                "bf16_gemm_3000x5000x4000"], _PAIR16),
+    ("f16", 129, INF, 1, INF, ["f16_gemm_8192", "f16_gemm_4096_relu"], _PAIR16),
+    ("w4a16", 1, 4, 1, INF, ["w4a16_gemm_m1"],
+     [{"path": "cuda_core", "ctas": c} for c in (128, 96)] + [{"path": "small_m"}] + _SMALL[2:]),
+    ("w4a16", 5, 128, 1, INF, ["w4a16_gemm_m16"], _SMALL),
+    ("w4a16", 129, INF, 1, INF, ["w4a16_gemm_m4096"],
+     [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
+    ("wfp4", 1, 128, 1, INF, ["wfp4_gemm_m1", "wfp4_gemm_m16"], _SMALL),
+    ("wfp4", 129, INF, 1, INF, ["wfp4_gemm_m4096"],
+     [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
+    ("f32_ffma", 1, 1024, 1, 1024, ["f32_ffma_gemm_1024"], [{"splits": k} for k in (1, 3, 4)]),
+    ("f32_tf32", 129, INF, 1, INF, ["f32_tf32_gemm_4096"], [{"group_m": g} for g in (8, 32)]),
+]
+SWEEP_MARGIN = 0.02
+TUNE_TABLE = os.path.join(ROOT, "tiled_dense_gemm_tma_b200", "csrc", "tune_table.h")
+SWEEP_REPORT = os.path.join(ROOT, "profiles", "tune_sweep.md")
+_RULE_FIELDS = ("op", "path", "m_lo", "m_hi", "n_lo", "n_hi", "ctas", "group_m", "splits",
+                "stages")
+
+
+def sweep_pick(times, margin=SWEEP_MARGIN):
+    """times: one list of per-workload seconds per candidate (candidate 0 is
+    the default).  Returns the index of the candidate with the smallest
+    geometric mean, or 0 unless it beats the default by more than margin."""
+    gm = [float(np.exp(np.mean(np.log(t)))) for t in times]
+    best = int(np.argmin(gm))
+    return best if gm[best] < gm[0] * (1.0 - margin) else 0
+
+
+def tune_table_source(rules, notes):
+    """C++ source of tune_table.h for the chosen rules (dicts of numbers)."""
+    lines = ["// tune_table.h -- built-in tuning rules (see tune.h).  Written by",
+             "// `python bench.py --sweep` on one B200 from the timings in",
+             "// profiles/tune_sweep.md; a class without a rule keeps every default.",
+             "#pragma once", '#include "tune.h"', "", "namespace tg {", "",
+             "constexpr TuneRule kBuiltinRules[] = {"]
+    for r, note in zip(rules, notes):
+        vals = ", ".join(("0x7fffffffffffffffll" if r[f] == INF else str(int(r[f])))
+                         for f in _RULE_FIELDS)
+        lines.append(f"    {{{vals}}},   // {note}")
+    lines += ["    {-1, 0, 0, 0, 0, 0, 0, 0, 0, 0},   // end: matches nothing", "};", "",
+              "}  // namespace tg", ""]
+    return "\n".join(lines)
+
+
+def run_sweep(args):
+    """Time every candidate of every class on this GPU; write the built-in
+    rules (tune_table.h) and the report (profiles/tune_sweep.md)."""
+    import torch
+    import tiled_dense_gemm_tma_b200 as tg
+    dev = torch.device("cuda", 0)
+    tg.load_library()
+    peaks, _ = load_peaks()
+    flush = (torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+             torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev),
+             torch.zeros((), dtype=torch.float32, device=dev))
+    chosen, notes = [], []
+    report = ["# Offline tile / stage sweep (tuning table)", "",
+              "Command: `python bench.py --sweep` on one B200.  Each candidate is timed",
+              f"as the median of {args.breakdown_iters} launches per workload, L2 flushed "
+              "before each launch; the default is the library's choice with no rule.  A class",
+              f"takes a rule when its best candidate's geometric-mean time is more than "
+              f"{SWEEP_MARGIN:.0%} below the default's.", ""]
+    tg.tune_set([])
+    for op, m_lo, m_hi, n_lo, n_hi, wls, cands in SWEEP_CLASSES:
+        cases = [Case(w, dev, peaks) for w in wls]
+        base = {"op": op, "m_lo": m_lo, "m_hi": m_hi, "n_lo": n_lo, "n_hi": n_hi}
+        allc = [{}] + list(cands)
+        times = []
+        for cand in allc:
+            tg.tune_set([dict(base, **cand)] if cand else [])
+            row = []
+            for c in cases:
+                med, _ = time_breakdown(c, args.breakdown_iters, 3, flush)
+                if tg.last_device_status() != 0:
+                    raise RuntimeError(f"device status after {op} {cand}")
+                row.append(med)
+            times.append(row)
+        tg.tune_set([])
+        best = sweep_pick(times)
+        cls = f"{op} M {m_lo}..{'inf' if m_hi == INF else m_hi}"
+        report += [f"## {cls}", "", "| candidate | " + " | ".join(f"{w} (us)" for w in wls) +
+                   " | geo-mean vs default |", "|---|" + "---|" * (len(wls) + 1)]
+        gm0 = float(np.exp(np.mean(np.log(times[0]))))
+        for i, (cand, row) in enumerate(zip(allc, times)):
+            gm = float(np.exp(np.mean(np.log(row))))
+            name = ", ".join(f"{k}={v}" for k, v in cand.items()) or "default"
+            mark = " **chosen**" if i == best else ""
+            report.append(f"| {name}{mark} | " + " | ".join(f"{t * 1e6:.2f}" for t in row) +
+                          f" | {gm / gm0:.3f} |")
+        report.append("")
+        if best:
+            r = {f: 0 for f in _RULE_FIELDS}
+            r.update(base)
+            r.update(allc[best])
+            r["op"] = tg.OPS[op]
+            r["path"] = tg.PATHS[r["path"]] if isinstance(r["path"], str) else r["path"]
+            chosen.append(r)
+            notes.append(f"{cls}: " + ", ".join(f"{k}={v}" for k, v in allc[best].items()) +
+                         f" ({float(np.exp(np.mean(np.log(times[best])))) / gm0:.3f} of the default)")
+        del cases
+        torch.cuda.empty_cache()
+    with open(TUNE_TABLE, "w") as f:
+        f.write(tune_table_source(chosen, notes))
+    with open(SWEEP_REPORT, "w") as f:
+        f.write("\n".join(report) + "\n")
+    print(json.dumps({"sweep": "done", "rules": len(chosen), "table": TUNE_TABLE,
+                      "report": SWEEP_REPORT}), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------- main
 
 def parse():
@@ -490,6 +617,8 @@ def parse():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown-iters", type=int, default=30)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the tuning table's candidates and rewrite its built-in rules")
     return ap.parse_args()
 
 
@@ -568,6 +697,8 @@ def main():
     ws, rank, local = dist_setup(args)
     if args.impl == "reference":
         return run_reference(args, ws, rank)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     torch.cuda.set_device(local)

@@ -230,6 +230,55 @@ TG_API tg_status tg_gemm_bf16_small_m_static(int64_t M, int64_t N, int64_t K,
                                              void *C, int64_t ldc,
                                              int epilogue, void *stream);
 
+/*
+ * Tuning table.  Every call picks its kernel family and launch shape from a
+ * table of rules keyed by operation and by ranges of M and N, the kernels
+ * being compiled ahead of time (this stands in for the parameter-space
+ * search of the pages' autotuner: "TileLang架构深度剖析", 自动调优系统; the
+ * tuning configuration of the gtnt.cn tutorial, section 3.3).  The built-in
+ * rules are written by the offline sweep `python bench.py --sweep`, which
+ * times the choices below on the device; rules installed with tg_tune_set
+ * are consulted before them.  The first rule with the call's op whose
+ * [m_lo, m_hi] holds M and [n_lo, n_hi] holds N applies; a field left 0
+ * keeps the library's default.  Transposed-operand calls, the fp32 FFMA
+ * kernel's tile shape and tg_gemm_bf16_small_m_static ignore the table.
+ */
+enum {
+    TG_OP_BF16 = 0, TG_OP_F16 = 1, TG_OP_W4A16 = 2, TG_OP_WFP4 = 3,
+    TG_OP_F32_FFMA = 4, TG_OP_F32_TF32 = 5
+};
+enum {
+    TG_PATH_AUTO = 0,       /* the default choice by M */
+    TG_PATH_CUDA_CORE = 1,  /* CUDA-core kernel: M <= 4 only; not for FP4 weights or fp32 */
+    TG_PATH_SMALL_M = 2,    /* weight-streaming tensor-core kernel: M <= 128 only */
+    TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit and 4-bit ops) */
+    TG_PATH_ONE_CTA = 4     /* persistent one-CTA tensor-core kernel (not fp32 FFMA) */
+};
+typedef struct {
+    int32_t op;             /* TG_OP_* */
+    int32_t path;           /* TG_PATH_*; must serve op and every M of the rule */
+    int64_t m_lo, m_hi;     /* inclusive range of M (>= 1) */
+    int64_t n_lo, n_hi;     /* inclusive range of N (>= 1) */
+    int32_t ctas;           /* persistent CTAs (CTA pairs for TG_PATH_CTA_PAIR); the
+                               stream-K split of the small-M and CUDA-core kernels;
+                               capped at the device's SMs; 0 = all */
+    int32_t group_m;        /* raster band height in (pair) tiles, 1..256; 0 = default */
+    int32_t splits;         /* TG_OP_F32_FFMA only: k ranges per output tile, 1..8 */
+    int32_t stages;         /* 16-bit CTA-pair kernel only: ring depth, 4 or 6 */
+} tg_tune_rule;
+
+/* Replace the run-time rules with `count` rules (at most 64; 0 clears them).
+ * A malformed rule -> TG_ERR_INVALID_ARG and the previous rules stay.  The
+ * rules apply to calls made after this returns, from any thread. */
+TG_API tg_status tg_tune_set(const tg_tune_rule *rules, int count);
+
+/* Copy up to `capacity` built-in rules to `out`; returns how many exist. */
+TG_API int tg_tune_builtin(tg_tune_rule *out, int capacity);
+
+/* The rule a call of operation `op` with these M and N would use (a rule of
+ * zero fields when none covers it); no CUDA call. */
+TG_API tg_status tg_tune_query(int op, int64_t M, int64_t N, tg_tune_rule *out);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 TG_API const char *tg_status_string(tg_status s);
 

@@ -237,3 +237,45 @@ def test_argument_validation_transposed(lib):
     assert _bf16_ex(lib, 64, 32, 16, 1, 1, lda=64, ldb=20) == ALIGN      # 40-byte B pitch
     assert _bf16_ex(lib, 0, 32, 16, 1, 1, lda=64, ldb=16) == OK          # empty output
     assert lib.tg_gemm_f16_ex(64, 32, 16, P, 60, 1, P, 32, 0, P, 32, 0, None) == INVALID
+
+
+def test_tuning_table_rules(lib):
+    """tg_tune_set validates every rule before installing any, run-time rules
+    are consulted before the built-in ones in the order given, and a call
+    shape no rule covers gets the all-default rule (no CUDA call needed)."""
+    from tiled_dense_gemm_tma_b200 import binding as b
+    b.tune_set([])
+    try:
+        builtin = b.tune_builtin()
+        for r in builtin:
+            assert b.tune_query(r["op"], r["m_lo"], r["n_lo"]) == r
+        rules = [{"op": "bf16", "path": "small_m", "m_lo": 5, "m_hi": 64, "ctas": 100},
+                 {"op": "bf16", "path": "cta_pair", "m_lo": 1, "m_hi": 1 << 40, "stages": 4,
+                  "group_m": 4},
+                 {"op": "f32_ffma", "splits": 3}]
+        b.tune_set(rules)
+        q = b.tune_query("bf16", 16, 8192)
+        assert (q["path"], q["ctas"]) == (b.PATHS["small_m"], 100)        # first match wins
+        q = b.tune_query("bf16", 65, 8192)
+        assert (q["path"], q["stages"], q["group_m"]) == (b.PATHS["cta_pair"], 4, 4)
+        assert b.tune_query("f32_ffma", 1024, 1024)["splits"] == 3
+        # malformed rules: nothing changes
+        bad = [{"op": "bf16", "path": "cuda_core", "m_hi": 5},       # CUDA-core kernel: M <= 4
+               {"op": "wfp4", "path": "cuda_core", "m_hi": 4},        # no CUDA-core FP4 kernel
+               {"op": "bf16", "path": "small_m", "m_hi": 129},        # small-M kernel: M <= 128
+               {"op": "f32_ffma", "path": "one_cta"},                 # fp32 FFMA has one kernel
+               {"op": "bf16", "splits": 2},                           # split count: FFMA only
+               {"op": "w4a16", "stages": 4},                          # ring depth: 16-bit pair only
+               {"op": "bf16", "stages": 5},
+               {"op": "bf16", "m_lo": 10, "m_hi": 9},
+               {"op": 9}, {"op": "bf16", "path": 7}, {"op": "bf16", "ctas": -1}]
+        for r in bad:
+            with pytest.raises(b.TgError):
+                b.tune_set([rules[0], r])
+            assert b.tune_query("bf16", 16, 8192)["ctas"] == 100
+        assert lib.tg_tune_set(None, 1) == INVALID
+        assert lib.tg_tune_set(None, 0) == OK
+        q = b.tune_query("bf16", 16, 8192)
+        assert q["ctas"] == 0 or q in builtin
+    finally:
+        b.tune_set([])

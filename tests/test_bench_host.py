@@ -101,3 +101,53 @@ def test_headline_sources_exist():
     csrc = os.path.join(ROOT, "tiled_dense_gemm_tma_b200", "csrc")
     for f in bench.HEADLINE_SOURCES:
         assert os.path.exists(os.path.join(csrc, f)), f
+
+
+def test_sweep_pick_needs_a_margin():
+    # candidate 0 is the default; a faster candidate wins only by more than 2 %
+    assert bench.sweep_pick([[1.0, 2.0], [0.99, 1.98]]) == 0
+    assert bench.sweep_pick([[1.0, 2.0], [0.99, 1.98], [0.5, 3.0]]) == 2
+    assert bench.sweep_pick([[1.0], [0.97]]) == 1
+
+
+def test_sweep_candidates_are_valid_rules():
+    """Every candidate the sweep can install is accepted by the library
+    (checked on the host: tg_tune_set validates without a device)."""
+    from tiled_dense_gemm_tma_b200 import binding as b, build as tg_build
+    tg_build.build()
+    try:
+        for op, m_lo, m_hi, n_lo, n_hi, wls, cands in bench.SWEEP_CLASSES:
+            for w in wls:
+                kind, M, N = bench.WORKLOADS[w][:3]
+                assert m_lo <= M <= m_hi and n_lo <= N <= n_hi, (op, w)
+            for cand in cands:
+                b.tune_set([dict({"op": op, "m_lo": m_lo, "m_hi": m_hi, "n_lo": n_lo,
+                                  "n_hi": n_hi}, **cand)])
+    finally:
+        b.tune_set([])
+
+
+def test_generated_tune_table_compiles(tmp_path):
+    """The sweep's C++ output compiles against tune.h and its rules read back."""
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("g++ not available")
+    rules = [{"op": 0, "path": 2, "m_lo": 5, "m_hi": 64, "n_lo": 1, "n_hi": bench.INF,
+              "ctas": 112, "group_m": 0, "splits": 0, "stages": 0},
+             {"op": 4, "path": 0, "m_lo": 1, "m_hi": 1024, "n_lo": 1, "n_hi": 1024,
+              "ctas": 0, "group_m": 0, "splits": 3, "stages": 0}]
+    (tmp_path / "tune_table.h").write_text(bench.tune_table_source(rules, ["a", "b"]))
+    (tmp_path / "main.cpp").write_text(
+        '#include <cstdio>\n#include "tune_table.h"\n'
+        'int main() { for (const auto& r : tg::kBuiltinRules) std::printf("%d %d %lld %lld %d %d\\n",'
+        ' r.op, r.path, (long long)r.m_lo, (long long)r.n_hi, r.ctas, r.splits); }\n')
+    csrc = os.path.join(ROOT, "tiled_dense_gemm_tma_b200", "csrc")
+    exe = tmp_path / "t"
+    subprocess.run([gxx, "-std=c++17", "-I", str(tmp_path), "-I", csrc, str(tmp_path / "main.cpp"),
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    assert out[0] == f"0 2 5 {bench.INF} 112 0"
+    assert out[1] == "4 0 1 1024 0 3"
+    assert out[2].startswith("-1 ")

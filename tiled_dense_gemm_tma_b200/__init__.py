@@ -14,4 +14,5 @@ from .binding import (  # noqa: F401
     TgError, gemm_f32, gemm_f16, gemm_bf16, gemm_w4a16, gemm_wfp4, gemm_bf16_small_m_static,
     matmul, last_device_status,
     lib_path, load_library, EPI_NONE, EPI_RELU, F32_FFMA, F32_TF32,
+    tune_set, tune_builtin, tune_query, OPS, PATHS,
 )

@@ -22,7 +22,21 @@ STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
 # Every symbol include/tg_gemm.h declares.
 EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16", "tg_gemm_wfp4",
            "tg_gemm_f16_ex", "tg_gemm_bf16_ex", "tg_gemm_bf16_small_m_static",
+           "tg_tune_set", "tg_tune_builtin", "tg_tune_query",
            "tg_status_string", "tg_last_device_status", "tg_num_sms")
+
+# Tuning table (include/tg_gemm.h: tg_tune_rule): operations and kernel paths.
+OPS = {"bf16": 0, "f16": 1, "w4a16": 2, "wfp4": 3, "f32_ffma": 4, "f32_tf32": 5}
+PATHS = {"auto": 0, "cuda_core": 1, "small_m": 2, "cta_pair": 3, "one_cta": 4}
+
+
+class TuneRule(ctypes.Structure):
+    """tg_tune_rule: which kernel family and launch shape a call uses."""
+    _fields_ = [("op", ctypes.c_int32), ("path", ctypes.c_int32),
+                ("m_lo", ctypes.c_int64), ("m_hi", ctypes.c_int64),
+                ("n_lo", ctypes.c_int64), ("n_hi", ctypes.c_int64),
+                ("ctas", ctypes.c_int32), ("group_m", ctypes.c_int32),
+                ("splits", ctypes.c_int32), ("stages", ctypes.c_int32)]
 
 _lib = None
 _lock = threading.Lock()
@@ -69,6 +83,12 @@ def load_library():
         lib.tg_last_device_status.argtypes = [vp]
         lib.tg_num_sms.argtypes = []
         lib.tg_num_sms.restype = ci
+        lib.tg_tune_set.argtypes = [ctypes.POINTER(TuneRule), ci]
+        lib.tg_tune_set.restype = ci
+        lib.tg_tune_builtin.argtypes = [ctypes.POINTER(TuneRule), ci]
+        lib.tg_tune_builtin.restype = ci
+        lib.tg_tune_query.argtypes = [ci, i64, i64, ctypes.POINTER(TuneRule)]
+        lib.tg_tune_query.restype = ci
         _lib = lib
         return lib
 
@@ -342,3 +362,45 @@ def gemm_bf16_small_m_static(A, B, C=None, relu=False, stream=None):
 def last_device_status(stream=None):
     """Synchronise the stream and return (and clear) the device status word."""
     return load_library().tg_last_device_status(_stream_handle(stream))
+
+
+_MAX_I64 = (1 << 63) - 1
+
+
+def _rule_of(d):
+    """A TuneRule from a dict: op and path by name or number, ranges default
+    to everything, knobs to 0 (the library's default)."""
+    op = OPS.get(d["op"], d["op"])
+    path = PATHS.get(d.get("path", 0), d.get("path", 0))
+    return TuneRule(op, path, d.get("m_lo", 1), d.get("m_hi", _MAX_I64), d.get("n_lo", 1),
+                    d.get("n_hi", _MAX_I64), d.get("ctas", 0), d.get("group_m", 0),
+                    d.get("splits", 0), d.get("stages", 0))
+
+
+def _dict_of(r):
+    return {f: getattr(r, f) for f, _ in TuneRule._fields_}
+
+
+def tune_set(rules):
+    """Install run-time tuning rules (list of dicts, see _rule_of), consulted
+    before the built-in ones; an empty list clears them."""
+    lib = load_library()
+    arr = (TuneRule * max(1, len(rules)))(*[_rule_of(d) for d in rules])
+    _check(lib.tg_tune_set(arr, len(rules)), "tg_tune_set")
+
+
+def tune_builtin():
+    """The built-in tuning rules, as dicts."""
+    lib = load_library()
+    n = lib.tg_tune_builtin(None, 0)
+    arr = (TuneRule * max(1, n))()
+    lib.tg_tune_builtin(arr, n)
+    return [_dict_of(arr[i]) for i in range(n)]
+
+
+def tune_query(op, M, N):
+    """The rule a call of `op` (name or number) with these M and N uses."""
+    lib = load_library()
+    r = TuneRule()
+    _check(lib.tg_tune_query(OPS.get(op, op), M, N, ctypes.byref(r)), "tg_tune_query")
+    return _dict_of(r)

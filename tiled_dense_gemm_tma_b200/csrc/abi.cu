@@ -82,6 +82,7 @@ tg::GemmArgs make_args(int64_t M, int64_t N, int64_t K, const void* A, int64_t l
     a.scales = nullptr; a.lds = 0; a.group = 0;
     a.relu = epilogue == TG_EPI_RELU;
     a.stream = stream;
+    a.path = a.ctas = a.group_m = a.splits = a.stages = 0;
     return a;
 }
 
@@ -102,7 +103,9 @@ tg_status tg_gemm_f32(int64_t M, int64_t N, int64_t K, const float* A, int64_t l
     tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 4);
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 4, stream);
-    tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
+    const tg::GemmArgs a = tg::with_rule(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream),
+                                         tg::tune_lookup(mode == TG_F32_TF32 ? tg::OP_F32_TF32
+                                                                             : tg::OP_F32_FFMA, M, N));
     return static_cast<tg_status>(mode == TG_F32_TF32 ? tg::launch_tc_tf32(a)
                                                       : tg::launch_ffma_f32(a));
 }
@@ -113,8 +116,8 @@ tg_status tg_gemm_f16(int64_t M, int64_t N, int64_t K, const void* A, int64_t ld
     tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2);
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    return static_cast<tg_status>(
-        tg::launch_tc_f16(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream)));
+    return static_cast<tg_status>(tg::launch_tc_f16(tg::with_rule(
+        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), tg::tune_lookup(tg::OP_F16, M, N))));
 }
 
 tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int trans_a,
@@ -123,8 +126,9 @@ tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t
     tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2, trans_a, trans_b);
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    return static_cast<tg_status>(tg::launch_tc_trans(
-        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), 0, trans_a, trans_b));
+    tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
+    if (!trans_a && !trans_b) a = tg::with_rule(a, tg::tune_lookup(tg::OP_F16, M, N));
+    return static_cast<tg_status>(tg::launch_tc_trans(a, 0, trans_a, trans_b));
 }
 
 tg_status tg_gemm_bf16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int trans_a,
@@ -133,8 +137,9 @@ tg_status tg_gemm_bf16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_
     tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2, trans_a, trans_b);
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    return static_cast<tg_status>(tg::launch_tc_trans(
-        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), 1, trans_a, trans_b));
+    tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
+    if (!trans_a && !trans_b) a = tg::with_rule(a, tg::tune_lookup(tg::OP_BF16, M, N));
+    return static_cast<tg_status>(tg::launch_tc_trans(a, 1, trans_a, trans_b));
 }
 
 tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
@@ -143,8 +148,8 @@ tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t l
     tg_status s = check_gemm(M, N, K, A, lda, B, ldb, C, ldc, epilogue, 2);
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    return static_cast<tg_status>(
-        tg::launch_tc_bf16(make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream)));
+    return static_cast<tg_status>(tg::launch_tc_bf16(tg::with_rule(
+        make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream), tg::tune_lookup(tg::OP_BF16, M, N))));
 }
 
 tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
@@ -166,7 +171,8 @@ tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K, const void* A, int64_t 
                   ldbq % 16 != 0 || (lds * 2) % 16 != 0))
         return TG_ERR_ALIGNMENT;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    tg::GemmArgs a = make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream);
+    tg::GemmArgs a = tg::with_rule(make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream),
+                                   tg::tune_lookup(tg::OP_W4A16, M, N));
     a.scales = scales;
     a.lds = lds;
     a.group = group_size;
@@ -192,7 +198,8 @@ tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K, const void* A, int64_t l
                   ldbq % 16 != 0 || lds % 16 != 0))
         return TG_ERR_ALIGNMENT;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
-    tg::GemmArgs a = make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream);
+    tg::GemmArgs a = tg::with_rule(make_args(M, N, K, A, lda, Bq, ldbq, C, ldc, epilogue, stream),
+                                   tg::tune_lookup(tg::OP_WFP4, M, N));
     a.scales = scales;
     a.lds = lds;
     a.group = block_size;

@@ -306,8 +306,14 @@ int launch_ffma_f32(const GemmArgs& a) {
     const long long tiles_n = (a.N + BN - 1) / BN, tiles_m = (a.M + BM - 1) / BM;
     const long long tiles = tiles_n * tiles_m;
     const long long kb_all = (a.K + BK - 1) / BK;
-    // Fewer output tiles than SMs: split K so the grid fills the chip.
-    const long long splits = ffma_splits(tiles, kb_all, di->num_sms);
+    // Fewer output tiles than SMs: split K so the grid fills the chip (or
+    // the tuning rule's split count, trimmed so that no k range is empty).
+    long long splits = ffma_splits(tiles, kb_all, di->num_sms);
+    if (a.splits > 0) {
+        const long long s = a.splits < kb_all ? a.splits : kb_all;
+        const long long per = (kb_all + s - 1) / s;
+        splits = (kb_all + per - 1) / per;
+    }
     int* tickets = nullptr;
     float* ws = nullptr;
     if (splits > 1 &&

@@ -13,6 +13,9 @@ using CfgF16 = TcCfg<2, 0, OutT::F16, 256, 4>;
 using CfgTF32 = TcCfg<4, 2, OutT::F32, 256, 4>;
 using Cfg2BF16 = Tc2Cfg<1, OutT::BF16, 6>;
 using Cfg2F16 = Tc2Cfg<0, OutT::F16, 6>;
+// a 4-slot ring, one of the ring depths the tuning table can choose
+using Cfg2BF16s4 = Tc2Cfg<1, OutT::BF16, 4>;
+using Cfg2F16s4 = Tc2Cfg<0, OutT::F16, 4>;
 // transposed operands (A stored K x M and/or B stored N x K)
 template <int FMT, OutT OUT>
 using Cfg2T10 = Tc2Cfg<FMT, OUT, 6, 1, 1>;
@@ -45,12 +48,13 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     const long long ntm = (a.M + Cfg::BM - 1) / Cfg::BM;
     const long long ntn = (a.N + Cfg::BN - 1) / Cfg::BN;
     const long long tiles = ntm * ntn;
-    const int grid = static_cast<int>(tiles < di->num_sms ? tiles : di->num_sms);
+    const int grid = static_cast<int>(persistent_grid(tiles, di->num_sms, a.ctas));
     TcParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
+    p.group_m = a.group_m > 0 ? a.group_m : Cfg::GROUP_M;
     p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
@@ -86,13 +90,13 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
         return kCudaError;
     const long long tiles = ((a.M + Cfg::PM - 1) / Cfg::PM) * ((a.N + Cfg::BN - 1) / Cfg::BN);
-    const long long pairs_max = di->num_sms / 2;
-    const int npairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
+    const int npairs = static_cast<int>(persistent_grid(tiles, di->num_sms / 2, a.ctas));
     TcParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
+    p.group_m = a.group_m > 0 ? a.group_m : Cfg::GROUP_M;
     p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
@@ -121,18 +125,33 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
 
 }  // namespace
 
+// The tuning rule's path (a.path) wins; by default M <= 4 takes the CUDA-core
+// kernel, M <= 128 the weight-streaming kernel, larger M the CTA-pair kernel
+// (the one-CTA kernel if a cluster launch is refused).
 int launch_tc_bf16(const GemmArgs& a) {
-    if (a.M <= kGemvMaxM) return launch_gemv_bf16(a);
-    if (a.M <= kSkinnyMaxM) return launch_skinny_bf16(a);
-    const int r = run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
-    if (r != kUnsupported) return r;
+    int path = a.path;
+    if (path == PATH_AUTO)
+        path = a.M <= kGemvMaxM ? PATH_CUDA_CORE : a.M <= kSkinnyMaxM ? PATH_SMALL_M : PATH_CTA_PAIR;
+    if (path == PATH_CUDA_CORE) return launch_gemv_bf16(a);
+    if (path == PATH_SMALL_M) return launch_skinny_bf16(a);
+    if (path == PATH_CTA_PAIR) {
+        const int r = a.stages == 4 ? run_pair<Cfg2BF16s4>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 54)
+                                    : run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
+        if (r != kUnsupported) return r;
+    }
     return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
 }
 int launch_tc_f16(const GemmArgs& a) {
-    if (a.M <= kGemvMaxM) return launch_gemv_f16(a);
-    if (a.M <= kSkinnyMaxM) return launch_skinny_f16(a);
-    const int r = run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
-    if (r != kUnsupported) return r;
+    int path = a.path;
+    if (path == PATH_AUTO)
+        path = a.M <= kGemvMaxM ? PATH_CUDA_CORE : a.M <= kSkinnyMaxM ? PATH_SMALL_M : PATH_CTA_PAIR;
+    if (path == PATH_CUDA_CORE) return launch_gemv_f16(a);
+    if (path == PATH_SMALL_M) return launch_skinny_f16(a);
+    if (path == PATH_CTA_PAIR) {
+        const int r = a.stages == 4 ? run_pair<Cfg2F16s4>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 55)
+                                    : run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
+        if (r != kUnsupported) return r;
+    }
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
 }
 // 16-bit GEMM with optionally transposed operands.  Only B transposed with

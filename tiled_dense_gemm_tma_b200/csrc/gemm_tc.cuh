@@ -75,6 +75,7 @@ struct TcParams {
     int M, N, K;
     int relu;
     int inject;               // debug: 1 = CTA 0's producer skips arming the first slot
+    int group_m;              // raster band height in tiles (tile_coords)
     unsigned long long timeout_ns;
     int* status;              // device status word (ST_TIMEOUT on an expired wait)
     void* C;                  // output base and row pitch (elements), for the ragged
@@ -256,7 +257,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int tm, tn;
-                tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+                tile_coords(t, ntm, ntn, p.group_m, tm, tn);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
@@ -335,7 +336,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t tl = 0, nstore = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
             int tm, tn;
-            tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+            tile_coords(t, ntm, ntn, p.group_m, tm, tn);
             const uint32_t acc = tl & 1;
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;

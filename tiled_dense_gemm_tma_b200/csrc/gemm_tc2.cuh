@@ -117,7 +117,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
                 int tm, tn;
-                tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+                tile_coords(t, ntm, ntn, p.group_m, tm, tn);
                 const int m0 = tm * Cfg::PM + rank * Cfg::BM;
                 const int n0 = tn * Cfg::BN + rank * Cfg::HN;
                 // boxes entirely past the matrix edge are not loaded: they only
@@ -221,7 +221,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t tl = 0, nstore = 0;
         for (int t = pair; t < num_tiles; t += npairs, ++tl) {
             int tm, tn;
-            tile_coords(t, ntm, ntn, Cfg::GROUP_M, tm, tn);
+            tile_coords(t, ntm, ntn, p.group_m, tm, tn);
             const uint32_t acc = tl & 1;
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;

@@ -131,7 +131,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int tm, tn;
-                tile_coords(t, ntm, ntn, W4::GROUP_M, tm, tn);
+                tile_coords(t, ntm, ntn, p.group_m, tm, tn);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const uint32_t s = it % W4::RAW_STAGES;
                     const uint32_t ph = (it / W4::RAW_STAGES) & 1;
@@ -201,7 +201,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t tl = 0, nstore = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
             int tm, tn;
-            tile_coords(t, ntm, ntn, W4::GROUP_M, tm, tn);
+            tile_coords(t, ntm, ntn, p.group_m, tm, tn);
             const uint32_t acc = tl & 1;
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
@@ -276,13 +276,14 @@ int run_large(const GemmArgs& a) {
         cudaSuccess)
         return kCudaError;
     const long long tiles = ((a.M + W4::BM - 1) / W4::BM) * ((a.N + W4::BN - 1) / W4::BN);
-    const int grid = static_cast<int>(tiles < di->num_sms ? tiles : di->num_sms);
+    const int grid = static_cast<int>(persistent_grid(tiles, di->num_sms, a.ctas));
     TcParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
     p.inject = inject_mode();
+    p.group_m = a.group_m > 0 ? a.group_m : W4::GROUP_M;
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;

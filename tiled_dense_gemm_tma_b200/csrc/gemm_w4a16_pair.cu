@@ -182,7 +182,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
                 int tm, tn;
-                tile_coords(t, ntm, ntn, W4P::GROUP_M, tm, tn);
+                tile_coords(t, ntm, ntn, p.group_m, tm, tn);
                 const int m0 = tm * W4P::PM + rank * W4P::BM;
                 const int n0 = tn * W4P::BN + rank * W4P::HN;
                 // A rows entirely past M are not loaded (never stored); packed
@@ -276,7 +276,7 @@ w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t tl = 0, nstore = 0;
         for (int t = pair; t < num_tiles; t += npairs, ++tl) {
             int tm, tn;
-            tile_coords(t, ntm, ntn, W4P::GROUP_M, tm, tn);
+            tile_coords(t, ntm, ntn, p.group_m, tm, tn);
             const uint32_t acc = tl & 1;
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
@@ -355,14 +355,14 @@ int run_pair(const GemmArgs& a) {
         cudaSuccess)
         return kCudaError;
     const long long tiles = ((a.M + W4P::PM - 1) / W4P::PM) * ((a.N + W4P::BN - 1) / W4P::BN);
-    const long long pairs_max = di->num_sms / 2;
-    const int npairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
+    const int npairs = static_cast<int>(persistent_grid(tiles, di->num_sms / 2, a.ctas));
     TcParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
     p.relu = a.relu;
     p.inject = inject_mode();
+    p.group_m = a.group_m > 0 ? a.group_m : W4P::GROUP_M;
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
     p.C = a.C;

@@ -403,7 +403,9 @@ int run_gemv(const GemmArgs& a) {
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
     SkPlan pl;
-    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK, di->num_sms, &pl)) return kUnsupported;
+    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK,
+                 static_cast<int>(persistent_grid(di->num_sms, di->num_sms, a.ctas)), &pl))
+        return kUnsupported;
     const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
     int* tickets = nullptr;
     float* ws = nullptr;

@@ -51,8 +51,10 @@ int* device_status_ptr();
 // `slot` (0..63) names the kernel in a per-device bitmask of done calls;
 // each kernel instantiation needs its own:
 //    0-4   gemm_tc.cu        one-CTA bf16/f16/tf32, CTA-pair bf16/f16
+//   54-55  gemm_tc.cu        CTA-pair bf16/f16 with a 4-slot ring (tuning table)
 //    5, 11-15 gemm_tc.cu     CTA-pair with transposed operands
 //    8     gemm_ffma.cu      9  gemm_w4a16.cu     10  gemm_w4a16_pair.cu
+//    6, 7  gemm_w4a16.cu, gemm_w4a16_pair.cu (FP4 weights)
 //   16-27  gemm_skinny.cu    28-35  gemm_skinny.cu (weights stored transposed)
 //   36-39  gemm_skinny.cu (FP4 weights)
 //   40-48  gemv.cu           50-53  gemm_skinny_static.cu

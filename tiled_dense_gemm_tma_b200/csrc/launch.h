@@ -3,6 +3,8 @@
 #pragma once
 #include <cstdint>
 
+#include "tune.h"
+
 namespace tg {
 
 // Internal status values; identical to the tg_status codes.
@@ -18,7 +20,30 @@ struct GemmArgs {
     int group;                       // 4-bit paths only
     int relu;
     void* stream;
+    // launch shape from the tuning table (tune.h); 0 = the launcher's default
+    int path;                        // TunePath: kernel family
+    int ctas;                        // persistent CTAs (CTA pairs), stream-K ranges
+    int group_m;                     // raster band height in tiles
+    int splits;                      // fp32 FFMA split-K ranges
+    int stages;                      // 16-bit CTA-pair ring depth (4 or 6)
 };
+
+// The arguments with a tuning rule's launch-shape fields.
+inline GemmArgs with_rule(GemmArgs a, const TuneRule& r) {
+    a.path = r.path;
+    a.ctas = r.ctas;
+    a.group_m = r.group_m;
+    a.splits = r.splits;
+    a.stages = r.stages;
+    return a;
+}
+
+// Persistent grid size: `units` of work over at most `cap` CTAs (the rule's
+// CTA count when set, else all of `cap`).
+inline long long persistent_grid(long long units, int cap, int ctas) {
+    const long long c = ctas > 0 && ctas < cap ? ctas : cap;
+    return units < c ? units : c;
+}
 
 int launch_tc_bf16(const GemmArgs& a);
 int launch_tc_f16(const GemmArgs& a);
