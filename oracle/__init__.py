@@ -9,7 +9,9 @@ triple loop on the gtnt.cn TileLang tutorial, section 1.1; C = A x B with
 row-major A and B on the mhpq.cn TileLang GEMM article, section 2.1; the
 ReLU post-processing and the dequantize GEMM on the blog.hotdry.top TileLang
 guide; the FP4-weight GEMM named on the krestaai TileLang architecture page,
-read as MXFP4 weights with bf16 activations).  The arithmetic lives in
+read as MXFP4 weights with bf16 activations; the 2:4 structured-sparse GEMM
+named on the blog.hotdry.top guide, read as the usual compressed values plus
+2-bit position codes).  The arithmetic lives in
 ``oracle.c``; this module only marshals
 numpy arrays through ctypes.
 
@@ -51,6 +53,11 @@ def _load():
         lib.oracle_gemm_wfp4.restype = None
         lib.oracle_dequant_fp4.argtypes = [i64, i64, vp, i64, vp, i64, i64, dp, i64]
         lib.oracle_dequant_fp4.restype = None
+        lib.oracle_expand_sp24.argtypes = [i64, i64, vp, i64, vp, i64, ctypes.c_int, dp, i64]
+        lib.oracle_expand_sp24.restype = None
+        lib.oracle_gemm_sp24.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ctypes.c_int,
+                                         dp, i64, ctypes.c_int]
+        lib.oracle_gemm_sp24.restype = None
         lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
         lib.oracle_e2m1_to_f64.restype = ctypes.c_double
         lib.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
@@ -195,6 +202,42 @@ def gemm_wfp4(A_bits, Bq, scales, N, block=32, relu=False):
     C = np.empty((M, N), np.float64)
     _load().oracle_gemm_wfp4(M, N, K, _ptr(A_bits), lda, _ptr(Bq), ldbq,
                              _ptr(scales), lds, block, _ptr(C), N, int(bool(relu)))
+    return C
+
+
+def _sp24_args(Ac, E, K, dtype):
+    if dtype not in ("f16", "bf16"):
+        raise ValueError("dtype must be 'f16' or 'bf16'")
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    ldac = _check2d(Ac, np.uint16, "Ac")
+    lde = _check2d(E, np.uint8, "E")
+    M = Ac.shape[0]
+    if E.shape[0] != M or Ac.shape[1] < K // 2 or E.shape[1] < (K + 7) // 8:
+        raise ValueError("Ac must be M x K/2 and E M x ceil(K/8)")
+    return M, ldac, lde, int(dtype == "bf16")
+
+
+def expand_sp24(Ac, E, K, dtype):
+    """Dense fp64 A (M x K) of a 2:4 compressed matrix: Ac (M x K/2 16-bit
+    bit patterns, the kept values of each chunk of 4 k) and E (M x K/8 bytes,
+    a 4-bit code per chunk: bits 0-1 / 2-3 = positions of the first / second
+    kept value; even chunk in the low nibble)."""
+    M, ldac, lde, bf = _sp24_args(Ac, E, K, dtype)
+    A = np.empty((M, K), np.float64)
+    _load().oracle_expand_sp24(M, K, _ptr(Ac), ldac, _ptr(E), lde, bf, _ptr(A), K)
+    return A
+
+
+def gemm_sp24(Ac, E, B_bits, dtype, relu=False):
+    """fp64 value of epi(A . B) for a 2:4 compressed A (see expand_sp24) and
+    a dense B (K x N) of the same 16-bit type, given as bit patterns."""
+    K, N = B_bits.shape
+    M, ldac, lde, bf = _sp24_args(Ac, E, K, dtype)
+    ldb = _check2d(B_bits, np.uint16, "B")
+    C = np.empty((M, N), np.float64)
+    _load().oracle_gemm_sp24(M, N, K, _ptr(Ac), ldac, _ptr(E), lde, _ptr(B_bits), ldb, bf,
+                             _ptr(C), N, int(bool(relu)))
     return C
 
 

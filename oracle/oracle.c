@@ -352,3 +352,56 @@ void oracle_round_bf16_n(const double *in, uint16_t *out, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(in[i]);
 }
+
+/* ------------------------------------------------------------------------ */
+/* 2:4 structured-sparse A.                                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The pages name a structured-sparse GEMM (T.gemm_sp, the 2:4 pattern, in the
+ * monitoring-and-debugging paragraph of "使用 Tilelang DSL 开发 GPU/CPU/加速器
+ * 高性能内核", blog.hotdry.top) and give no storage format; the library's
+ * reading is the usual 2:4 compressed form of a row-major M x K matrix A:
+ *   - each row is cut into chunks of 4 consecutive k (chunk c: k in
+ *     [4c, 4c + 4)); at most two entries of a chunk are non-zero;
+ *   - Ac (M x K/2) holds, for chunk c, its two kept values in positions
+ *     2c and 2c + 1 (first, second);
+ *   - E (M rows of K/8 bytes) holds a 4-bit code per chunk, chunk c in byte
+ *     c / 2 (low nibble for even c, high nibble for odd c); bits 0-1 of the
+ *     code give the position inside the chunk of the first kept value, bits
+ *     2-3 that of the second.
+ * Expansion to the dense matrix, in double: A[i][4c + idx_p] receives
+ * Ac[i][2c + p] for p = 0, 1; every other entry is zero.  (A code naming one
+ * position twice adds both values there: the plain reading.)  K is a
+ * multiple of 4.
+ */
+void oracle_expand_sp24(int64_t M, int64_t K, const uint16_t *Ac, int64_t ldac,
+                        const uint8_t *E, int64_t lde, int bf16, double *A, int64_t lda)
+{
+    for (int64_t i = 0; i < M; ++i) {
+        double *arow = A + i * lda;
+        for (int64_t k = 0; k < K; ++k) arow[k] = 0.0;
+        for (int64_t c = 0; c < K / 4; ++c) {
+            int code = oracle_code4(E + i * lde, c);
+            for (int p = 0; p < 2; ++p) {
+                int idx = (code >> (2 * p)) & 3;
+                uint16_t bits = Ac[i * ldac + 2 * c + p];
+                double v = bf16 ? oracle_bf16_to_f64(bits) : oracle_f16_to_f64(bits);
+                arow[4 * c + idx] += v;
+            }
+        }
+    }
+}
+
+/* Expand A, then the plain GEMM with B (K x N) of the same 16-bit type. */
+void oracle_gemm_sp24(int64_t M, int64_t N, int64_t K,
+                      const uint16_t *Ac, int64_t ldac, const uint8_t *E, int64_t lde,
+                      const uint16_t *B, int64_t ldb, int bf16,
+                      double *C, int64_t ldc, int relu)
+{
+    double *A = (double *)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * (size_t)(K > 0 ? K : 1));
+    oracle_expand_sp24(M, K, Ac, ldac, E, lde, bf16, A, K);
+    gemm_generic(M, N, K, A, K, load_f64, B, ldb, bf16 ? load_bf16 : load_f16, C, ldc, relu);
+    free(A);
+}
+

@@ -33,6 +33,8 @@ CASES = {
     "w4a16_130x300x384_seed4": lambda: synth.w4a16(130, 300, 384, 4),
     "wfp4_16x8192x8192_seed4": lambda: synth.wfp4(16, 8192, 8192, 4),
     "wfp4_130x300x384_seed4": lambda: synth.wfp4(130, 300, 384, 4),
+    "sp24_bf16_300x520x640_seed2": lambda: synth.sp24(300, 520, 640, 2, "bf16"),
+    "sp24_f16_16x4096x4096_seed3": lambda: synth.sp24(16, 4096, 4096, 3, "f16"),
 }
 
 

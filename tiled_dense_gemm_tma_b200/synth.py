@@ -146,3 +146,40 @@ def with_ld(X, ld):
     out = np.zeros((R, ld), X.dtype)
     out[:, :C] = X
     return out[:, :C]
+
+
+# The six increasing position pairs (i0 < i1) a chunk of 4 can keep.
+SP24_PAIRS = ((0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3))
+
+
+def sp24(M, N, K, seed, dtype="bf16", scale_by_sqrt_k=True, a_int=None):
+    """Inputs of the 2:4 structured-sparse GEMM (sparse A, dense B).
+
+    Each chunk of 4 consecutive k of a row of A keeps two positions, a pair
+    drawn uniformly from the six increasing pairs.  Returns (Ac 16-bit bits
+    M x K/2: the kept values in increasing k; E uint8 M x ceil(K/8): position
+    codes, i0 | i1 << 2 per chunk, even chunk in the low nibble; B bits
+    K x N; pos int M x K/2: the k of each kept value).  Kept values are
+    N(0, 1) / sqrt(K / 2) (or integers in [-a_int, a_int]); B is
+    N(0, 1) / sqrt(K).  K must be a multiple of 4.
+    """
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    rng = np.random.default_rng(seed)
+    C4 = K // 4
+    which = rng.integers(0, 6, size=(M, C4))
+    if a_int is None:
+        s = 1.0 / math.sqrt(max(K // 2, 1)) if scale_by_sqrt_k else 1.0
+        vals = rng.standard_normal(size=(M, K // 2)) * s
+    else:
+        vals = rng.integers(-a_int, a_int + 1, size=(M, K // 2)).astype(np.float64)
+    sb = 1.0 / math.sqrt(K) if (scale_by_sqrt_k and K > 0) else 1.0
+    B = rng.standard_normal(size=(K, N)) * sb if a_int is None else \
+        rng.integers(-a_int, a_int + 1, size=(K, N)).astype(np.float64)
+    pairs = np.array(SP24_PAIRS, np.int64)[which]            # M x C4 x 2
+    codes = (pairs[..., 0] | (pairs[..., 1] << 2)).astype(np.uint8)
+    E = pack_nibbles(codes) if C4 else np.zeros((M, 0), np.uint8)
+    base = (4 * np.arange(C4))[None, :, None]
+    pos = (base + pairs).reshape(M, K // 2)
+    return store(vals, dtype), E, store(B, dtype), pos
+
