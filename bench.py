@@ -67,6 +67,9 @@ WORKLOADS = {
     "wfp4_gemm_m1": ("wfp4", 1, 8192, 8192, 4, False, "wfp4"),
     "wfp4_gemm_m16": ("wfp4", 16, 8192, 8192, 4, False, "wfp4"),
     "wfp4_gemm_m4096": ("wfp4", 4096, 8192, 8192, 4, False, "wfp4"),
+    # 2:4 structured-sparse A (two kept values per chunk of 4 k, N(0,1)/sqrt(K/2);
+    # the six position pairs uniform), dense B N(0,1)/sqrt(K)
+    "sp24_bf16_gemm_8192": ("sp24_bf16", 8192, 8192, 8192, 2, False, "sp24"),
 }
 # Transposed-operand variants: name -> (workload, A stored K x M, B stored N x K).
 # The same seeded matrices, stored transposed in HBM.
@@ -104,6 +107,9 @@ def make_inputs(name):
     if kind == "wfp4":
         A, Bq, E, _ = synth.wfp4(M, N, K, seed)
         return {"A": A, "Bq": Bq, "S": E}
+    if kind == "sp24_bf16":
+        Ac, E, B, _ = synth.sp24(M, N, K, seed, "bf16")
+        return {"A": Ac, "E": E, "B": B}
     st = {"bf16": "bf16", "f16": "f16"}.get(kind, "f32")
     if dist == "normal_sqrtk":
         A, B = synth.normal(M, N, K, seed, st, scale_by_sqrt_k=True)
@@ -154,11 +160,18 @@ def workload_facts(name, peaks):
     MMA work and dequantisation arithmetic are not counted.  A contraction
     whose flops per byte lie below the ridge (tensor peak / HBM bandwidth)
     is HBM-bound; the fp32 FFMA path is bound by the FMA pipe ("alu"); TF32
-    takes the bf16 peak times the nominal dense ratio 1.1 / 2.25."""
+    takes the bf16 peak times the nominal dense ratio 1.1 / 2.25.  The 2:4
+    sparse GEMM counts the multiply-adds its kept values need (M*N*K flops,
+    half the dense count) and the compressed A (K/2 values and K/8 code
+    bytes per row), against the dense bf16 peak: the sparse tensor cores do
+    the same multiply-adds per cycle on half the operands."""
     base = TRANSPOSED.get(name, (name, False, False))[0]
     kind, M, N, K = WORKLOADS[base][:4]
     flops = 2.0 * M * N * K
-    if kind == "w4a16":
+    if kind == "sp24_bf16":
+        flops = float(M) * N * K
+        alg_bytes = M * (K // 2) * 2 + M * ((K + 7) // 8) + K * N * 2 + M * N * 2
+    elif kind == "w4a16":
         alg_bytes = M * K * 2 + K * ((N + 1) // 2) + (K // 128) * N * 2 + M * N * 2
     elif kind == "wfp4":
         alg_bytes = M * K * 2 + K * ((N + 1) // 2) + ((K + 31) // 32) * N + M * N * 2
@@ -201,6 +214,14 @@ class Case:
             self.dtype = "f16 x int4"
             self._host = host
             self.run = lambda: tg.gemm_w4a16(self.A, self.Bq, self.S, N, C=self.C, relu=relu)
+        elif kind == "sp24_bf16":
+            self.A = _torch_of(host["A"], "bf16", device)
+            self.E = _torch_of(host["E"], "u8", device)
+            self.B = _torch_of(host["B"], "bf16", device)
+            self.C = _empty_out(M, N, torch.bfloat16, device)
+            self.dtype = "bf16 (A 2:4 sparse)"
+            self._host = host
+            self.run = lambda: tg.gemm_sp24(self.A, self.E, self.B, C=self.C, relu=relu)
         elif kind == "wfp4":
             self.A = _torch_of(host["A"], "bf16", device)
             self.Bq = _torch_of(host["Bq"], "u8", device)
@@ -236,6 +257,11 @@ class Case:
     def host_pinned(self):
         """Pinned host copies of the inputs and a pinned host output (e2e)."""
         import torch
+        if self.kind == "sp24_bf16":
+            pairs = [(self.A, _torch_of(self._host["A"], "bf16", "cpu", pinned=True)),
+                     (self.E, _torch_of(self._host["E"], "u8", "cpu", pinned=True)),
+                     (self.B, _torch_of(self._host["B"], "bf16", "cpu", pinned=True))]
+            return pairs, _empty_out(self.M, self.N, self.C.dtype, "cpu", pinned=True)
         if self.kind in ("w4a16", "wfp4"):
             ak, sk = ("f16", "f16") if self.kind == "w4a16" else ("bf16", "u8")
             hA = _torch_of(self._host["A"], ak, "cpu", pinned=True)
@@ -454,6 +480,13 @@ def oracle_block(name, host, rows, cols):
         t0 = time.perf_counter()
         fn(A, Bq, S, N=ncols)
         return time.perf_counter() - t0
+    if kind == "sp24_bf16":
+        Ac = np.ascontiguousarray(host["A"][rows])
+        E = np.ascontiguousarray(host["E"][rows])
+        B = np.ascontiguousarray(host["B"][:, cols])
+        t0 = time.perf_counter()
+        oracle.gemm_sp24(Ac, E, B, "bf16")
+        return time.perf_counter() - t0
     A = np.ascontiguousarray(host["A"][rows])
     B = np.ascontiguousarray(host["B"][:, cols])
     fn = {"bf16": oracle.gemm_bf16, "f16": oracle.gemm_f16}.get(kind, oracle.gemm_f32)
@@ -489,19 +522,22 @@ def oracle_rate(name, host, budget_s):
 INF = (1 << 63) - 1
 _PAIR16 = ([{"path": "cta_pair", "stages": st, "group_m": g} for st in (4, 6) for g in (4, 8, 16)] +
            [{"path": "one_cta", "group_m": g} for g in (8, 16)])
-_SMALL = [{"path": "small_m", "ctas": c} for c in (140, 128, 112, 96, 74)]
+_SMALL = [{"path": "small_m", "ctas": c} for c in (140, 128, 120, 112, 104, 96, 74)]
+# (the small-M classes are measured on wide weight matrices only, so their
+# rules cover N >= 4096; narrower N keeps the defaults)
 SWEEP_CLASSES = [
-    ("bf16", 5, 64, 1, INF, ["bf16_gemm_16x8192x8192"], _SMALL + [{"path": "cta_pair"}]),
-    ("bf16", 65, 128, 1, INF, ["bf16_gemm_128x14336x4096"], _SMALL + [{"path": "cta_pair"}]),
+    ("bf16", 5, 64, 4096, INF, ["bf16_gemm_16x8192x8192"], _SMALL + [{"path": "cta_pair"}]),
+    ("bf16", 65, 128, 4096, INF, ["bf16_gemm_128x14336x4096"], _SMALL + [{"path": "cta_pair"}]),
     ("bf16", 129, INF, 1, INF, ["bf16_gemm_8192", "bf16_gemm_4096", "bf16_gemm_8192x1024x8192",
                                 "bf16_gemm_3000x5000x4000"], _PAIR16),
     ("f16", 129, INF, 1, INF, ["f16_gemm_8192", "f16_gemm_4096_relu"], _PAIR16),
-    ("w4a16", 1, 4, 1, INF, ["w4a16_gemm_m1"],
-     [{"path": "cuda_core", "ctas": c} for c in (128, 96)] + [{"path": "small_m"}] + _SMALL[2:]),
-    ("w4a16", 5, 128, 1, INF, ["w4a16_gemm_m16"], _SMALL),
+    ("w4a16", 1, 4, 4096, INF, ["w4a16_gemm_m1"],
+     [{"path": "cuda_core", "ctas": c} for c in (136, 128, 120, 96)] + [{"path": "small_m"}] +
+     _SMALL[2:]),
+    ("w4a16", 5, 128, 4096, INF, ["w4a16_gemm_m16"], _SMALL),
     ("w4a16", 129, INF, 1, INF, ["w4a16_gemm_m4096"],
      [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
-    ("wfp4", 1, 128, 1, INF, ["wfp4_gemm_m1", "wfp4_gemm_m16"], _SMALL),
+    ("wfp4", 1, 128, 4096, INF, ["wfp4_gemm_m1", "wfp4_gemm_m16"], _SMALL),
     ("wfp4", 129, INF, 1, INF, ["wfp4_gemm_m4096"],
      [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
     ("f32_ffma", 1, 1024, 1, 1024, ["f32_ffma_gemm_1024"], [{"splits": k} for k in (1, 3, 4)]),

@@ -21,8 +21,8 @@
  * - Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
  *   current CUDA device.  The caller owns every buffer.  C must not overlap
  *   A, B or the scales (not checked).
- * - Leading dimensions are in elements (in bytes for packed 4-bit weights
- *   and E8M0 scale bytes), and must be >= the row length.
+ * - Leading dimensions are in elements (in bytes for packed 4-bit weights,
+ *   E8M0 scale bytes and 2:4 position codes), and must be >= the row length.
  * - stream is a cudaStream_t passed as void*; NULL means the legacy default
  *   stream.  Calls are asynchronous: they validate, enqueue and return.
  * - Sizes: M, N, K >= 0.  M == 0 or N == 0 -> TG_OK, nothing is launched.
@@ -205,6 +205,40 @@ TG_API tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K,
                        const uint8_t *scales, int64_t lds, int block_size,
                        void *C, int64_t ldc,
                        int epilogue, void *stream);
+
+/*
+ * tg_gemm_sp24_f16, tg_gemm_sp24_bf16 -- 2:4 structured-sparse GEMM (the
+ * structured-sparse T.gemm_sp with the 2:4 pattern of the blog.hotdry.top
+ * TileLang guide, monitoring-and-debugging paragraph; the pages give no
+ * format, this library defines it):  C = epi(A . B) where A (M x K) keeps at
+ * most two non-zeros in every chunk of 4 consecutive k of a row and is
+ * passed compressed:
+ *   Ac:  M x K/2 fp16 / bf16 values, row pitch ldac (elements, % 8 == 0):
+ *        the two kept values of chunk c (k in [4c, 4c + 4)) at columns 2c
+ *        and 2c + 1, the first before the second.
+ *   E:   M rows of ceil(K/8) code bytes, row pitch lde in BYTES (% 16 == 0):
+ *        a 4-bit code per chunk, chunk c in byte c/2 (low nibble for even c);
+ *        bits 0-1 give the position (0-3) inside the chunk of the first kept
+ *        value, bits 2-3 that of the second.  Positions should be distinct
+ *        (a chunk with fewer non-zeros keeps zeros at unused positions).
+ *   B:   K x N dense, row pitch ldb (elements, % 8 == 0); C: M x N, ldc.
+ * K must be a multiple of 4 (else TG_ERR_UNSUPPORTED).  Runs on the sparse
+ * tensor cores (tcgen05.mma.sp) with fp32 accumulation and one rounding of
+ * each result to C's type.  Same status and ownership rules as
+ * tg_gemm_f16.
+ */
+TG_API tg_status tg_gemm_sp24_f16(int64_t M, int64_t N, int64_t K,
+                           const void *Ac, int64_t ldac,
+                           const uint8_t *E, int64_t lde,
+                           const void *B, int64_t ldb,
+                           void *C, int64_t ldc,
+                           int epilogue, void *stream);
+TG_API tg_status tg_gemm_sp24_bf16(int64_t M, int64_t N, int64_t K,
+                            const void *Ac, int64_t ldac,
+                            const uint8_t *E, int64_t lde,
+                            const void *B, int64_t ldb,
+                            void *C, int64_t ldc,
+                            int epilogue, void *stream);
 
 /*
  * tg_gemm_bf16_small_m_static -- tg_gemm_bf16 for M <= 128 that never

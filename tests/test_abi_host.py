@@ -103,6 +103,21 @@ def test_argument_validation_wfp4(lib):
     assert w(4, 32, 256, P, 256, P, 1 << 40, P, 32, 32, P, 32, 0, None) == UNSUP
 
 
+def test_argument_validation_sp24(lib):
+    for f in (lib.tg_gemm_sp24_f16, lib.tg_gemm_sp24_bf16):
+        # M, N, K, Ac, ldac, E, lde (bytes), B, ldb, C, ldc, epi, stream
+        assert f(8, 8, 30, P, 16, P, 16, P, 8, P, 8, 0, None) == UNSUP        # K % 4
+        assert f(8, 8, 64, P, 24, P, 16, P, 8, P, 8, 0, None) == INVALID      # ldac < K/2
+        assert f(8, 8, 256, P, 128, P, 16, P, 8, P, 8, 0, None) == INVALID    # lde < K/8
+        assert f(8, 8, 64, P, 36, P, 16, P, 8, P, 8, 0, None) == ALIGN        # 72-byte pitch
+        assert f(8, 8, 64, P, 32, P, 24, P, 8, P, 8, 0, None) == ALIGN        # lde % 16
+        assert f(8, 8, 64, P, 32, None, 16, P, 8, P, 8, 0, None) == INVALID
+        assert f(8, 8, 64, P, 32, P + 4, 16, P, 8, P, 8, 0, None) == ALIGN
+        assert f(0, 8, 64, P, 32, P, 16, P, 8, P, 8, 0, None) == OK
+        assert f(8, 8, 64, P, 32, P, 16, P, 8, P, 8, 3, None) == INVALID
+        assert f(8, 8, 64, P, 32, P, (1 << 62) + 16, P, 8, P, 8, 0, None) == UNSUP
+
+
 def test_row_pitch_limits(lib):
     """Row pitches of 2^40 bytes or more are refused before any product
     ld * sizeof(element) is formed, so even pitches near 2^63 are reported
@@ -166,6 +181,7 @@ def test_valid_calls_without_a_device_report_no_device(lib):
         assert lib.tg_gemm_f32(64, 64, 64, P, 64, P, 64, P, 64, 0, mode, None) == NODEV
     assert lib.tg_gemm_w4a16(4, 32, 256, P, 256, P, 16, P, 32, 128, P, 32, 0, None) == NODEV
     assert lib.tg_gemm_wfp4(4, 32, 200, P, 200, P, 16, P, 32, 32, P, 32, 0, None) == NODEV
+    assert lib.tg_gemm_sp24_bf16(8, 8, 64, P, 32, P, 16, P, 8, P, 8, 0, None) == NODEV
     assert lib.tg_gemm_bf16_ex(64, 64, 64, P, 64, 1, P, 64, 1, P, 64, 0, None) == NODEV
     assert lib.tg_gemm_f16_ex(64, 64, 64, P, 64, 0, P, 64, 1, P, 64, 0, None) == NODEV
     assert lib.tg_gemm_bf16_small_m_static(16, 64, 64, P, 64, P, 64, P, 64, 0, None) == NODEV

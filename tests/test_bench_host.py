@@ -43,6 +43,9 @@ EXPECTED = {
     "wfp4_gemm_m1": (0.1342, 35.68, "hbm"),
     "wfp4_gemm_m16": (2.147, 36.18, "hbm"),
     "wfp4_gemm_m4096": (549.8, 169.9, "tensor"),
+    # 2:4 sparse A: M*N*K flops (kept values only); Ac 67.1 MB + codes 8.4 MB
+    # + B 134.2 MB + C 134.2 MB
+    "sp24_bf16_gemm_8192": (549.8, 343.9, "tensor"),
 }
 
 

@@ -7,9 +7,10 @@ library, so no call allocates.
 Called through the C ABI on two calls in a row and checked three ways:
 against the fp64 oracle at the bf16 tolerance (rtol = atol = 1e-2, relative
 Frobenius error <= 1e-2); against tg_gemm_bf16 bit for bit where both run
-the same weight-streaming kernel (5 <= M <= 128: same plan, same summation
-order), and within the tolerance where tg_gemm_bf16 takes its CUDA-core
-kernel (M <= 4); and that a call on a stream the library has never seen
+the same weight-streaming kernel with the same plan (5 <= M <= 128, the
+regular call held to the small-M kernel on all SMs by a tuning rule: same
+summation order), and within the tolerance where tg_gemm_bf16 takes its
+CUDA-core kernel (M <= 4); and that a call on a stream the library has never seen
 leaves the device's free memory unchanged.  Also checks the size limits.
 
 This file is named to be collected last, so that a run stopping at the
@@ -61,8 +62,15 @@ def test_matches_oracle_and_regular_entry_point_twice(lib, shape, relu):
     ref = oracle.gemm_bf16(A, B, relu)
     dA, dB = to_dev(A, "bf16"), to_dev(B, "bf16")
     _, C_reg, _ = guarded_out(M, N, "bf16")
-    assert _call(lib, "tg_gemm_bf16", dA, dB, C_reg, relu) == TG_OK
-    torch.cuda.synchronize()
+    # the regular call on the small-M kernel with its default plan (all SMs),
+    # whatever the tuning table would choose for this shape
+    import tiled_dense_gemm_tma_b200 as tg
+    tg.tune_set([{"op": "bf16", "path": "small_m", "m_lo": 5, "m_hi": 128}] if M >= 5 else [])
+    try:
+        assert _call(lib, "tg_gemm_bf16", dA, dB, C_reg, relu) == TG_OK
+        torch.cuda.synchronize()
+    finally:
+        tg.tune_set([])
     regular = from_dev(C_reg, "bf16")
     for _ in range(2):
         big, C, pad = guarded_out(M, N, "bf16")

@@ -22,6 +22,7 @@ STATUS = {0: "TG_OK", 1: "TG_ERR_INVALID_ARG", 2: "TG_ERR_ALIGNMENT",
 # Every symbol include/tg_gemm.h declares.
 EXPORTS = ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16", "tg_gemm_wfp4",
            "tg_gemm_f16_ex", "tg_gemm_bf16_ex", "tg_gemm_bf16_small_m_static",
+           "tg_gemm_sp24_f16", "tg_gemm_sp24_bf16",
            "tg_tune_set", "tg_tune_builtin", "tg_tune_query",
            "tg_status_string", "tg_last_device_status", "tg_num_sms")
 
@@ -72,6 +73,9 @@ def load_library():
         for name in ("tg_gemm_w4a16", "tg_gemm_wfp4"):
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, ci,
                                            vp, i64, ci, vp]
+        for name in ("tg_gemm_sp24_f16", "tg_gemm_sp24_bf16"):
+            getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, i64, vp, i64, ci, vp]
+            getattr(lib, name).restype = ci
         for name in ("tg_gemm_f16_ex", "tg_gemm_bf16_ex"):
             getattr(lib, name).argtypes = [i64, i64, i64, vp, i64, ci, vp, i64, ci, vp, i64, ci, vp]
         for name in ("tg_gemm_f32", "tg_gemm_f16", "tg_gemm_bf16", "tg_gemm_w4a16",
@@ -340,6 +344,42 @@ def gemm_wfp4(A, Bq, scales, N, C=None, block_size=32, relu=False, stream=None):
                                 C.data_ptr(), _ld(C, "C"), EPI_RELU if relu else EPI_NONE,
                                 _stream_handle(stream))
     _check(code, "tg_gemm_wfp4")
+    return C
+
+
+def gemm_sp24(Ac, E, B, C=None, relu=False, stream=None):
+    """C = epi(A @ B) for a 2:4 structured-sparse A given compressed.
+
+    Ac: M x K/2 float16 or bfloat16 (the two kept values of every chunk of 4
+    consecutive k, in increasing k); E: M x ceil(K/8) uint8 position codes
+    (per chunk 4 bits, bits 0-1 / 2-3 = positions of the first / second kept
+    value, even chunk in the low nibble); B: K x N of Ac's dtype.  K is taken
+    from B and must be a multiple of 4.
+    """
+    import torch
+    lib = load_library()
+    if Ac.dtype not in (torch.float16, torch.bfloat16) or B.dtype != Ac.dtype:
+        raise TypeError("Ac and B must be float16 or bfloat16, the same")
+    if E.dtype != torch.uint8:
+        raise TypeError("E must be uint8")
+    if Ac.dim() != 2 or E.dim() != 2 or B.dim() != 2:
+        raise ValueError("Ac, E and B must be 2-D")
+    K, N = B.shape
+    M = Ac.shape[0]
+    if Ac.shape[1] != K // 2 or E.shape[0] != M or E.shape[1] < (K + 7) // 8:
+        raise ValueError("Ac must be M x K/2 and E M x ceil(K/8)")
+    _require_cuda(Ac.device, (Ac, "Ac"), (E, "E"), (B, "B"))
+    if C is None:
+        C = empty_out(M, N, Ac.dtype, Ac.device)
+    elif C.shape != (M, N) or C.dtype != Ac.dtype:
+        raise ValueError("C has the wrong shape or dtype")
+    _require_cuda(Ac.device, (C, "C"))
+    name = "tg_gemm_sp24_bf16" if Ac.dtype == torch.bfloat16 else "tg_gemm_sp24_f16"
+    with _device_ctx(Ac):
+        code = getattr(lib, name)(M, N, K, Ac.data_ptr(), _ld(Ac, "Ac"), E.data_ptr(), _ld(E, "E"),
+                                  B.data_ptr(), _ld(B, "B"), C.data_ptr(), _ld(C, "C"),
+                                  EPI_RELU if relu else EPI_NONE, _stream_handle(stream))
+    _check(code, name)
     return C
 
 

@@ -206,6 +206,46 @@ tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K, const void* A, int64_t l
     return static_cast<tg_status>(tg::launch_wfp4(a));
 }
 
+namespace {
+
+// 2:4 sparse A: Ac (M x K/2 values), E (M x ceil(K/8) code bytes), B (K x N).
+tg_status sp24(int64_t M, int64_t N, int64_t K, const void* Ac, int64_t ldac, const uint8_t* E,
+               int64_t lde, const void* B, int64_t ldb, void* C, int64_t ldc, int epilogue,
+               void* stream, int bf16) {
+    if (M < 0 || N < 0 || K < 0) return TG_ERR_INVALID_ARG;
+    if (epilogue != TG_EPI_NONE && epilogue != TG_EPI_RELU) return TG_ERR_INVALID_ARG;
+    if (K % 4 != 0) return TG_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return TG_OK;
+    if (!C || ldc < N) return TG_ERR_INVALID_ARG;
+    if (K > 0 && (!Ac || !E || !B || ldac < K / 2 || lde < (K + 7) / 8 || ldb < N))
+        return TG_ERR_INVALID_ARG;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return TG_ERR_UNSUPPORTED;
+    if (!pitch_ok(ldc, 2) ||
+        (K > 0 && (!pitch_ok(ldac, 2) || !pitch_ok(lde, 1) || !pitch_ok(ldb, 2))))
+        return TG_ERR_UNSUPPORTED;
+    if (!aligned16(C) || (ldc * 2) % 16 != 0) return TG_ERR_ALIGNMENT;
+    if (K > 0 && (!aligned16(Ac) || !aligned16(E) || !aligned16(B) || (ldac * 2) % 16 != 0 ||
+                  lde % 16 != 0 || (ldb * 2) % 16 != 0))
+        return TG_ERR_ALIGNMENT;
+    if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
+    const tg::GemmArgs a = make_args(M, N, K, Ac, ldac, B, ldb, C, ldc, epilogue, stream);
+    return static_cast<tg_status>(tg::launch_sp24(a, E, lde, bf16));
+}
+
+}  // namespace
+
+tg_status tg_gemm_sp24_f16(int64_t M, int64_t N, int64_t K, const void* Ac, int64_t ldac,
+                           const uint8_t* E, int64_t lde, const void* B, int64_t ldb, void* C,
+                           int64_t ldc, int epilogue, void* stream) {
+    return sp24(M, N, K, Ac, ldac, E, lde, B, ldb, C, ldc, epilogue, stream, 0);
+}
+
+tg_status tg_gemm_sp24_bf16(int64_t M, int64_t N, int64_t K, const void* Ac, int64_t ldac,
+                            const uint8_t* E, int64_t lde, const void* B, int64_t ldb, void* C,
+                            int64_t ldc, int epilogue, void* stream) {
+    return sp24(M, N, K, Ac, ldac, E, lde, B, ldb, C, ldc, epilogue, stream, 1);
+}
+
 const char* tg_status_string(tg_status s) {
     switch (s) {
         case TG_OK: return "TG_OK";

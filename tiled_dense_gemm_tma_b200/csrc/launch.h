@@ -58,6 +58,8 @@ int launch_wfp4(const GemmArgs& a);
 int launch_wfp4_large(const GemmArgs& a);
 int launch_wfp4_pair(const GemmArgs& a);
 int launch_skinny_wfp4(const GemmArgs& a);
+// 2:4 sparse A: a.A / a.lda are the compressed values, E / lde the codes.
+int launch_sp24(const GemmArgs& a, const void* E, int64_t lde, int bf16);
 int launch_skinny_bf16(const GemmArgs& a);
 int launch_skinny_f16(const GemmArgs& a);
 int launch_skinny_w4a16(const GemmArgs& a);

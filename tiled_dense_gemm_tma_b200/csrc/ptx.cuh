@@ -226,6 +226,32 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 lanes x 4 consecutive 32-bit columns: thread t of the warp writes lane
+// (base_lane + t), columns [col, col + 4).
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Sparse D(tmem) (+)= A(smem, 2:4 compressed along K) x B(smem), kind::f16,
+// K = 32 (dense) per instruction; `e_tmem` is the TMEM address of the
+// metadata (even column), idesc carries the sparse flag and which of the two
+// columns holds this instruction's metadata.  No output lane is disabled.
+__device__ __forceinline__ void mma_f16_sp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate, uint32_t e_tmem) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%5], %3, {%6, %6, %6, %6}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem), "r"(0u)
+        : "memory");
+}
+
 // ------------------------------------------------------- UMMA descriptors
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
@@ -249,7 +275,9 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo,
     return d;
 }
 
-// Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.
+// Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation
+// (dense; a sparse MMA sets bit 2 and puts the metadata column selector in
+// bits 0-1).
 //   fmt: 0 = f16, 1 = bf16, 2 = tf32 (A and B alike)
 //   a_mn / b_mn: 1 if that operand is MN-major in shared memory.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t m, uint32_t n,
