@@ -152,4 +152,49 @@ long long check_ffma_splits(int max_tiles, int max_kb, int num_sms, long long* c
     return bad;
 }
 
+// cl_split returns the largest admissible split S (none larger qualifies),
+// or 0 exactly when no admissible split fills three quarters of the SMs;
+// its cluster ranges tile [0, KB) with none empty.
+static bool cl_admissible(long long T, long long KB, int gn, long long cap, int max_s, int S) {
+    return S <= max_s && S <= KB && gn % (32 * S) == 0 && T * S <= cap;
+}
+
+long long check_cl_split(long long* checked) {
+    long long bad = 0, n = 0;
+    const int gns[] = {128, 256};
+    const int smss[] = {1, 7, 132, 148};
+    const int max_ss[] = {1, 2, 8};
+    for (long long T = 1; T <= 300; ++T) for (long long KB = 1; KB <= 40; ++KB)
+    for (int gn : gns) for (int sms : smss) for (int max_s : max_ss) {
+        const long long caps[] = {sms, 2ll * sms, 128};
+        for (long long cap : caps) {
+            const int S = tg::cl_split(T, KB, gn, cap, sms, max_s);
+            ++n;
+            if (S != 0 && S != 1 && S != 2 && S != 4 && S != 8) { ++bad; continue; }
+            int best = 0;
+            for (int c = 8; c >= 1; c >>= 1)
+                if (cl_admissible(T, KB, gn, cap, max_s, c)) { best = c; break; }
+            const bool fills = best && T * best * 4 >= 3ll * sms;
+            ++n; bad += S != (fills ? best : 0);
+            if (S) {
+                int next = 0;
+                for (int r = 0; r < S; ++r) {
+                    const int b = tg::cl_begin(r, int(KB), S), e = tg::cl_begin(r + 1, int(KB), S);
+                    ++n; bad += b != next || e <= b;
+                    next = e;
+                }
+                ++n; bad += next != KB;
+            }
+        }
+    }
+    // the shapes the weight-streaming kernels meet most
+    ++n; bad += tg::cl_split(32, 128, 256, 148, 148, 8) != 4;     // 4-bit weights, N = 8192
+    ++n; bad += tg::cl_split(64, 64, 128, 148, 148, 8) != 2;      // 16-bit weights, N = 8192
+    ++n; bad += tg::cl_split(112, 32, 128, 148, 148, 8) != 1;     // 16-bit, N = 14336: whole groups
+    ++n; bad += tg::cl_split(256, 64, 128, 148, 148, 8) != 0;     // more groups than SMs
+    ++n; bad += tg::cl_split(20, 64, 128, 148, 148, 8) != 0;      // 80 CTAs at most: stream-K
+    *checked = n;
+    return bad;
+}
+
 }  // extern "C"

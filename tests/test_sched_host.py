@@ -1,7 +1,8 @@
 """Host checks of the kernels' work-distribution arithmetic (csrc/tile_sched.h).
 
 The stream-K ranges of the weight-streaming kernels, their launch plan (how
-many split-K partial slots a column group needs), the grouped raster of the
+many split-K partial slots a column group needs), the split-K-in-a-cluster
+plan that replaces stream-K where it fills the GPU, the grouped raster of the
 persistent tile kernels and the fp32 split-K ranges are plain integer
 arithmetic shared by the device code and the launchers.  A wrong range here
 drops or double-counts part of the k sum, or leaves tiles unwritten, on some
@@ -32,7 +33,8 @@ def chk(tmp_path_factory):
                        ("check_stream_k_large", []),
                        ("check_sk_plan", []),
                        ("check_tile_coords", [ctypes.c_int, ctypes.c_int]),
-                       ("check_ffma_splits", [ctypes.c_int, ctypes.c_int, ctypes.c_int])):
+                       ("check_ffma_splits", [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+                       ("check_cl_split", [])):
         fn = getattr(lib, name)
         fn.argtypes = args + [ctypes.POINTER(ll)]
         fn.restype = ll
@@ -68,4 +70,9 @@ def test_tile_raster_is_a_banded_bijection(chk):
 @pytest.mark.parametrize("num_sms", [148, 132, 1])
 def test_fp32_split_k_ranges(chk, num_sms):
     bad, n = _run(chk.check_ffma_splits, 300, 600, num_sms)
+    assert n > 100_000 and bad == 0
+
+
+def test_cluster_split_plan(chk):
+    bad, n = _run(chk.check_cl_split)
     assert n > 100_000 and bad == 0

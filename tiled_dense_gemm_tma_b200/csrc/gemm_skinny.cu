@@ -1,5 +1,6 @@
 // gemm_skinny.cu -- launchers of the weight-streaming (small-M) kernel, for
-// B stored K x N (the plain call) or N x K (a transposed-B call); its split-K
+// B stored K x N (the plain call) or N x K (a transposed-B call).  Split-K
+// runs inside clusters where that fills the GPU; otherwise stream-K, whose
 // partials and tile tickets live in the per-stream workspace (workspace.cu).
 #include "gemm_skinny.cuh"
 #include "host.cuh"
@@ -15,14 +16,23 @@ int run(const GemmArgs& a) {
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
+    const long long cap = persistent_grid(di->num_sms, di->num_sms, a.ctas);
     SkPlan pl;
-    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK,
-                 static_cast<int>(persistent_grid(di->num_sms, di->num_sms, a.ctas)), &pl))
-        return kUnsupported;
-    const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
+    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK, static_cast<int>(cap), &pl)) return kUnsupported;
+    auto kern = skinny_kernel<Cfg>;
+    const int mi = MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3;
+    const int slot = W == WKind::FP4 ? 36 + mi
+                   : WK ? 28 + static_cast<int>(W) * 4 + mi : 16 + static_cast<int>(W) * 4 + mi;
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return kCudaError;
+    // split-K inside clusters where T groups x a small split fill the GPU
+    // (no workspace, no tickets), else stream-K over the stream's workspace
+    const int S = skinny_cluster_split<Cfg>(pl.T, pl.KB, cap, di->num_sms, slot);
+    const long long T = pl.T, KB = pl.KB, U = pl.U, J = pl.J;
+    const long long G = S ? T * S : pl.G;
     int* tickets = nullptr;
     float* ws = nullptr;
-    if (!stream_workspace(dev, a.stream, T, T * J * MPAD * Cfg::GN * 4, &tickets, &ws))
+    if (!S && !stream_workspace(dev, a.stream, T, T * J * MPAD * Cfg::GN * 4, &tickets, &ws))
         return kCudaError;
 
     CUtensorMap tW, tS, tX;
@@ -59,12 +69,6 @@ int run(const GemmArgs& a) {
     if (!tensor_map_2d(&tX, a.A, xt, 2, a.K, a.M, a.lda * 2, 64, MPAD, SWZ_128))
         return kCudaError;
 
-    auto kern = skinny_kernel<Cfg>;
-    const int mi = MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3;
-    const int slot = W == WKind::FP4 ? 36 + mi
-                   : WK ? 28 + static_cast<int>(W) * 4 + mi : 16 + static_cast<int>(W) * 4 + mi;
-    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
-        return kCudaError;
     SkParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
@@ -74,6 +78,7 @@ int run(const GemmArgs& a) {
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.S = S;
     p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
@@ -82,9 +87,8 @@ int run(const GemmArgs& a) {
     p.ws = ws;
     p.tickets = tickets;
     if (!p.status) return kCudaError;
-    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(
-        tW, tS, tX, p);
-    return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
+    return skinny_launch<Cfg>(G, S, static_cast<cudaStream_t>(a.stream), tW, tS, tX, p) == cudaSuccess
+               ? kOk : kCudaError;
 }
 
 template <WKind W, int WK = 0>

@@ -23,6 +23,15 @@
 //   group's last segment (counted with an atomic ticket) sums the partials
 //   in segment order -- deterministic -- applies ReLU, rounds and writes C,
 //   and resets the ticket for the next call.
+// * Split-K inside clusters (16-bit weights, where T groups times a split S
+//   in {8, 4, 2, 1} fill at least three quarters of the SMs): group t goes to
+//   the S CTAs of cluster t, each taking a contiguous part of its k-units.
+//   When its accumulator is final a CTA's ring is idle; the ranks exchange
+//   "ring free" signals, write their partials of each rank's GN/S columns
+//   into that rank's ring through distributed shared memory, and each rank
+//   sums its columns' S partials in rank order (deterministic) and writes C.
+//   No global round trips (partials, fences, tickets) sit between the last
+//   MMA and the output, which is where stream-K spends its tail.
 // * Weights arrive either as fp16/bf16 tiles by TMA, or as packed 4-bit
 //   weights + scales that converter warps expand (dequant.cuh): signed
 //   integers with fp16 group scales into fp16 tiles, or FP4 (E2M1) codes
@@ -30,7 +39,8 @@
 #pragma once
 #include "ptx.cuh"
 #include "dequant.cuh"
-#include "tile_sched.h"     // sk_begin / sk_owner
+#include "tile_sched.h"     // sk_begin / sk_owner / cl_begin / cl_split
+#include "host.cuh"         // max_active_clusters
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -90,6 +100,11 @@ struct SkCfg {
     // 6-warp 16-bit kernel than beside the 4-bit converters)
     static constexpr int RED_ROWS = Q4 ? 2 : 8;
     static constexpr int THREADS = 32 * (2 + EPI_WARPS + CONV_WARPS);
+    // Split-K inside a cluster: a CTA's ring, idle once its accumulator is
+    // final, receives the partials of the columns it owns from every rank
+    // ([rank][MPAD rows][GN/S columns] fp32, MPAD x GN floats in all).
+    static constexpr int RING_BYTES = RAW_STAGES * RAW_SLOT;
+    static constexpr bool CL_OK = MPAD * GN * 4 <= RING_BYTES;
     // Independent accumulator sets: k-step kk of a unit accumulates into set
     // kk % R, so consecutive small MMAs do not wait on each other's result;
     // the epilogue adds the R sets in a fixed order.
@@ -120,6 +135,8 @@ struct SkParams {
     int relu;
     int T, KB, U;             // column groups (GN wide), k-slices per group, units = T * KB
     int J;                    // workspace slots per tile (max segments of a tile)
+    int S;                    // 0: stream-K (ws, tickets); S >= 1: column group blockIdx.x / S
+                              // split over the S CTAs of one cluster (1: whole groups)
     int inject;               // debug: 1 = CTA 0's producer skips arming the first slot
     unsigned long long timeout_ns;
     int* status;
@@ -188,7 +205,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     uint64_t* drain = tempty + 2;
     uint64_t* epi_bar = drain + 1;                                   // epilogue warps joined
     uint64_t* flag_bar = epi_bar + 1;                                // ticket result published
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(flag_bar + 1);
+    uint64_t* cl_ready = flag_bar + 1;                               // peers' rings may receive
+    uint64_t* cl_full = cl_ready + 1;                                // this CTA's columns arrived
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cl_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;
 
@@ -202,10 +221,19 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     const int lane = threadIdx.x & 31;
     const int G = gridDim.x;
     const int c = blockIdx.x;
-    const int u0 = sk_begin(c, p.U, G);
-    const int u1 = sk_begin(c + 1, p.U, G);
     const int KB = p.KB;
+    int u0, u1, crank = 0;                   // crank: rank in the cluster
+    if (p.S) {
+        const int tg0 = c / p.S;
+        crank = c - tg0 * p.S;
+        u0 = tg0 * KB + cl_begin(crank, KB, p.S);
+        u1 = tg0 * KB + cl_begin(crank + 1, KB, p.S);
+    } else {
+        u0 = sk_begin(c, p.U, G);
+        u1 = sk_begin(c + 1, p.U, G);
+    }
     const uint64_t limit = p.timeout_ns;
+    bool cl_waited = false;                  // this thread passed the start-up cluster barrier
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
@@ -224,6 +252,8 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
         mbar_init(drain, 1);
         mbar_init(epi_bar, Cfg::EPI_WARPS);
         mbar_init(flag_bar, 1);
+        mbar_init(cl_ready, p.S > 1 ? p.S - 1 : 1);
+        mbar_init(cl_full, Cfg::EPI_WARPS * Cfg::NSUB);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -237,6 +267,10 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Peers arrive on this CTA's barriers only after a cluster barrier whose
+    // arrive is here (after the barriers are initialised); each thread waits
+    // on it before its first remote arrive, or at the end.
+    if (p.S > 1) cluster_arrive_release();
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
@@ -398,6 +432,25 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             const uint32_t acc = seg & 1;
             if (!bounded_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, limit, p.status)) break;
             tc_fence_after();
+            // Split-K in a cluster: the accumulator is final, so every unit
+            // has been consumed and this CTA's ring is idle.  Once the peers'
+            // barriers exist, tell the peers their partials of this CTA's
+            // columns may come, and wait until every peer's ring may take
+            // this CTA's partials of its columns.
+            const bool cl = p.S > 1 && !whole;
+            const int CW = Cfg::GN / (p.S > 1 ? p.S : 1);   // columns a rank owns
+            if (cl) {
+                cluster_wait_acquire();
+                cl_waited = true;
+                if (etid == 0) {
+                    // the copy engine's and the tensor core's accesses to the
+                    // ring are complete; the peers' plain stores come next
+                    fence_proxy_async_smem();
+                    for (int pr = 0; pr < p.S; ++pr)
+                        if (pr != crank) mbar_arrive_relaxed_cluster(mapa_shared(smem_u32(cl_ready), pr));
+                }
+                if (!bounded_wait_cluster(cl_ready, 0, abort_flag, limit, p.status)) break;
+            }
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    acc * Cfg::ACC_COLS;
             // Partials are stored m-major (row m of GN fp32 per slot): the 32
@@ -405,7 +458,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
             // each reducer load covers whole 128-byte lines.
             const long long sstride = static_cast<long long>(Cfg::MPAD) * Cfg::GN;
             float* slot = nullptr;
-            if (!whole) {
+            if (!whole && !cl) {
                 const int jseg = c - sk_owner(t * KB, p.U, G);
                 slot = p.ws + (static_cast<long long>(t) * p.J + jseg) * sstride;
             }
@@ -436,6 +489,14 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                             const float x = __uint_as_float(v[i]);
                             if (n < p.N) store_out<Cfg::OUTW>(p.C, p.ldc, m, n, p.relu ? fmaxf(x, 0.f) : x);
                         }
+                    } else if (cl) {
+                        // into the owner's ring: [this rank][row m][column - o*CW]
+                        const int o = nj / CW;
+                        const uint32_t dst = mapa_shared(
+                            smem_u32(ring) + static_cast<uint32_t>(((crank * Cfg::MPAD + mc) * CW + nj - o * CW) * 4), o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (mc + i < p.M) st_shared_cluster_f32(dst + i * CW * 4, __uint_as_float(v[i]));
                     } else {
                         float* col = slot + nj;
 #pragma unroll
@@ -444,10 +505,48 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                     }
                 }
             }
+            if (cl) {
+                // the warp's 32 columns of sub-tile j belong to one owner:
+                // one fence for all the warp's stores, one arrive per sub-tile
+                fence_acq_rel_cluster();
+                __syncwarp();
+                if (lane == 0)
+#pragma unroll
+                    for (int j = 0; j < Cfg::NSUB; ++j)
+                        mbar_arrive_release_cluster(
+                            mapa_shared(smem_u32(cl_full), (j * Cfg::TN + q * 32) / CW));
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
             if (whole) continue;
+            if (cl) {
+                // Owner: every (warp, sub-tile) slice of this rank's columns
+                // from every rank, summed in rank order (deterministic).
+                if (!bounded_wait_cluster(cl_full, 0, abort_flag, limit, p.status)) break;
+                // CW is 32, 64 or 128 columns: thread etid takes the 4
+                // neighbouring columns 4 * (etid % (CW / 4)) of rows
+                // etid / (CW / 4), + 512 / CW, ...
+                const float4* buf = reinterpret_cast<const float4*>(ring);
+                const int lg = __ffs(CW >> 2) - 1;                 // log2(CW / 4)
+                const int c4 = etid & ((CW >> 2) - 1);
+                const int n = t * Cfg::GN + crank * CW + 4 * c4;
+                for (int m = etid >> lg; m < p.M; m += (32 * Cfg::EPI_WARPS) >> lg) {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+                        if (r < p.S) {
+                            const float4 v4 = buf[((r * Cfg::MPAD + m) << lg) + c4];
+                            x.x += v4.x; x.y += v4.y; x.z += v4.z; x.w += v4.w;
+                        }
+                    float o[4] = {x.x, x.y, x.z, x.w};
+                    if (p.relu)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o[e] = fmaxf(o[e], 0.f);
+                    store_out4<Cfg::OUTW>(p.C, p.ldc, m, n, p.N, o);
+                }
+                continue;
+            }
             // Publish the partial, take a ticket; the tile's last contributor
             // reduces.  The epilogue warps meet on mbarriers with bounded waits
             // (never an unbounded bar.sync, which a warp that gave up would hang).
@@ -561,6 +660,57 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
+    if (p.S > 1) {
+        // no CTA leaves while a peer may still write into its shared memory
+        if (!cl_waited) cluster_wait_acquire();
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
+}
+
+// Host side, shared by the regular and the static entry points.  The
+// cluster split of cl_split for T column groups of KB k-units, lowered until
+// the device holds all T clusters of that size at once; 0 selects stream-K.
+// 4-bit weights always take stream-K: their pace is set per SM (expanding
+// the packed weights), so they need every SM, which the split into T*S CTAs
+// seldom gives.  `slot` is the kernel's attribute slot (set_smem_attr done).
+template <class Cfg>
+inline int skinny_cluster_split(long long T, long long KB, long long cap, int num_sms, int slot) {
+    if constexpr (!Cfg::CL_OK || Cfg::Q4) {
+        return 0;
+    } else {
+        const void* k = reinterpret_cast<const void*>(skinny_kernel<Cfg>);
+        int max_s = 8;
+        for (;;) {
+            const int S = cl_split(T, KB, Cfg::GN, cap, num_sms, max_s);
+            if (S <= 1) return S;
+            if (max_active_clusters(k, slot, S, Cfg::THREADS, Cfg::SMEM_BYTES) >= T) return S;
+            max_s = S / 2;
+        }
+    }
+}
+
+// Launch G CTAs; clusters of S CTAs when S > 1 (p.S == S).
+template <class Cfg>
+inline cudaError_t skinny_launch(long long G, int S, cudaStream_t stream, const CUtensorMap& tW,
+                                 const CUtensorMap& tS, const CUtensorMap& tX, const SkParams& p) {
+    if (S > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
+        cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, skinny_kernel<Cfg>, tW, tS, tX, p);
+    }
+    skinny_kernel<Cfg><<<static_cast<unsigned>(G), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tW, tS, tX, p);
+    return cudaGetLastError();
 }
 
 }  // namespace tg

@@ -1,7 +1,8 @@
 // gemm_skinny_static.cu -- tg_gemm_bf16_small_m_static: the small-M bf16 GEMM
-// (weight-streaming, stream-K kernel of gemm_skinny.cuh) with its scratch
-// memory in a fixed array of device memory that is part of the library
-// image, so a call never allocates.
+// (the weight-streaming kernel of gemm_skinny.cuh) with its scratch memory in
+// a fixed array of device memory that is part of the library image, so a call
+// never allocates.  Shapes whose split-K runs inside clusters need no scratch
+// at all; the others use the array for their stream-K partials.
 //
 // Who needs this: code that may not call cudaMalloc / cudaFree at the point
 // where it runs the GEMM -- for example a program whose memory pool has
@@ -16,14 +17,17 @@
 //   (4096) tile tickets.  The CUDA runtime places the arrays in device memory
 //   of every GPU on which this part of the library is loaded (at the latest
 //   on the first call there) and keeps them until the process exits.  Shapes
-//   whose partials or tiles exceed that return TG_ERR_UNSUPPORTED.
+//   that take stream-K and whose partials or tiles exceed that return
+//   TG_ERR_UNSUPPORTED.
 // - Every call uses the same array.  Tickets are cleared at the start of each
 //   call; partials are overwritten before they are read.  Calls that overlap
 //   on the GPU (different streams, or different host threads on one device)
 //   race on the array and give wrong results: serialise them.
 // - Set-up: the first call on each device looks up the array's device address
 //   with cudaGetSymbolAddress (the array's name in host code is only a host
-//   stand-in) and caches it; make that first call before any stream capture.
+//   stand-in) and how many clusters of the kernel the device holds at once
+//   (cudaOccupancyMaxActiveClusters), and caches both; make that first call
+//   before any stream capture.
 #include "gemm_skinny.cuh"
 #include "host.cuh"
 #include "launch.h"
@@ -100,22 +104,28 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     using Cfg = SkCfg<WKind::BF16, MPAD>;
     SkPlan pl;
     if (!sk_plan(N, K, Cfg::GN, Cfg::BK, di->num_sms, &pl)) return TG_ERR_UNSUPPORTED;
-    const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
-    if (T > kStaticTickets || T * J * MPAD * Cfg::GN > kStaticPartialFloats)
-        return TG_ERR_UNSUPPORTED;                     // beyond the fixed scratch size
-    float* part = nullptr;
-    int* tick = nullptr;
-    if (!static_scratch(dev, &part, &tick)) return TG_ERR_CUDA;
-    CUtensorMap tW, tX;
-    if (!encode_map(&tW, B, N, K, ldb * 2, 64, Cfg::BK)) return TG_ERR_CUDA;
-    if (!encode_map(&tX, A, K, M, lda * 2, 64, MPAD)) return TG_ERR_CUDA;
     auto kern = skinny_kernel<Cfg>;
     const int slot = 50 + (MPAD == 16 ? 0 : MPAD == 32 ? 1 : MPAD == 64 ? 2 : 3);
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
         return TG_ERR_CUDA;
+    // the plan of tg_gemm_bf16 on all SMs: split-K inside clusters (no
+    // scratch) where that fills the GPU, else stream-K over the fixed arrays
+    const int S = skinny_cluster_split<Cfg>(pl.T, pl.KB, di->num_sms, di->num_sms, slot);
+    const long long T = pl.T, KB = pl.KB, U = pl.U, J = pl.J;
+    const long long G = S ? T * S : pl.G;
+    float* part = nullptr;
+    int* tick = nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(tick, 0, static_cast<size_t>(T) * sizeof(int), s) != cudaSuccess)
-        return TG_ERR_CUDA;
+    if (!S) {
+        if (T > kStaticTickets || T * J * MPAD * Cfg::GN > kStaticPartialFloats)
+            return TG_ERR_UNSUPPORTED;                 // beyond the fixed scratch size
+        if (!static_scratch(dev, &part, &tick)) return TG_ERR_CUDA;
+        if (cudaMemsetAsync(tick, 0, static_cast<size_t>(T) * sizeof(int), s) != cudaSuccess)
+            return TG_ERR_CUDA;
+    }
+    CUtensorMap tW, tX;
+    if (!encode_map(&tW, B, N, K, ldb * 2, 64, Cfg::BK)) return TG_ERR_CUDA;
+    if (!encode_map(&tX, A, K, M, lda * 2, 64, MPAD)) return TG_ERR_CUDA;
     SkParams p;
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
@@ -125,6 +135,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.S = S;
     p.inject = 0;
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
@@ -133,8 +144,7 @@ tg_status run_static(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda
     p.ws = part;
     p.tickets = tick;
     if (!p.status) return TG_ERR_CUDA;
-    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(tW, tW, tX, p);
-    return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_CUDA;
+    return skinny_launch<Cfg>(G, S, s, tW, tW, tX, p) == cudaSuccess ? TG_OK : TG_ERR_CUDA;
 }
 
 }  // namespace

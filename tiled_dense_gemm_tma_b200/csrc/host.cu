@@ -155,4 +155,44 @@ cudaError_t set_smem_attr(const void* func, int bytes, int slot) {
     return e;
 }
 
+namespace {
+// -1: not asked yet; indexed [device][slot][log2 S - 1]
+std::atomic<int> g_max_clusters[kMaxDevices][64][3];
+std::once_flag g_max_clusters_once;
+}  // namespace
+
+int max_active_clusters(const void* func, int slot, int S, int threads, int smem_bytes) {
+    std::call_once(g_max_clusters_once, [] {
+        for (auto& d : g_max_clusters)
+            for (auto& sl : d)
+                for (auto& v : sl) v.store(-1, std::memory_order_relaxed);
+    });
+    int dev = 0;
+    const int si = S == 2 ? 0 : S == 4 ? 1 : S == 8 ? 2 : -1;
+    if (si < 0 || slot < 0 || slot >= 64 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
+        dev >= kMaxDevices)
+        return 0;
+    std::atomic<int>& cached = g_max_clusters[dev][slot][si];
+    int n = cached.load(std::memory_order_acquire);
+    if (n >= 0) return n;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, func, &cfg) != cudaSuccess) {
+        cudaGetLastError();                        // clear: treated as "no clusters"
+        n = 0;
+    }
+    cached.store(n, std::memory_order_release);
+    return n;
+}
+
 }  // namespace tg

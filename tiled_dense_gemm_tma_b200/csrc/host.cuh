@@ -61,4 +61,10 @@ int* device_status_ptr();
 //   56-57  gemm_sp24.cu
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 
+// Clusters of S CTAs (threads and dynamic shared memory bytes each) of the
+// kernel in attribute slot `slot` that the current device holds at once
+// (cudaOccupancyMaxActiveClusters), cached per device, slot and S; 0 if the
+// query fails.  The slot's shared-memory attribute must be set first.
+int max_active_clusters(const void* func, int slot, int S, int threads, int smem_bytes);
+
 }  // namespace tg

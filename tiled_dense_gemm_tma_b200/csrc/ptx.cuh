@@ -141,6 +141,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Ampere-style asynchronous 16-byte copy global -> shared (L2 only), and the
+// wait for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -324,6 +334,67 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cl_addr, 
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+
+// ------------------------------------------- split-K reduction in a cluster
+//
+// Partial sums travel between the CTAs of a cluster through distributed
+// shared memory: plain stores to a peer's shared memory, then an arrive on an
+// mbarrier of that peer with release semantics at cluster scope; the peer
+// waits with acquire semantics at cluster scope and then reads the data.
+
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t cl_addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cl_addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
+// Arrive with no ordering of this thread's earlier accesses (a pure signal).
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
+// bounded_wait for a barrier that peers of the cluster arrive on.
+__device__ __forceinline__ bool bounded_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort, uint64_t limit_ns,
+                                                     int* status) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_acq_cluster(bar, parity, 1000000u)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            atomicExch(status, ST_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// The two halves of a cluster-wide barrier, per thread (not warp-aligned):
+// every thread of every CTA of the cluster arrives once per phase and waits
+// before it arrives again.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // Tiled 2-D TMA load into this CTA's shared memory whose completion is

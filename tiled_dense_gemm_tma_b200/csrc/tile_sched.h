@@ -74,6 +74,30 @@ inline bool sk_plan(long long N, long long K, int gn, int bk, int num_sms, SkPla
     return true;
 }
 
+// ------------------------------------------------- split-K inside a cluster
+// The alternative to stream-K when T column groups times a small split S
+// fill the GPU: group t goes to the S CTAs of cluster t, and rank r of the
+// cluster takes the k-units [t*KB + cl_begin(r), t*KB + cl_begin(r + 1)).
+// The ranks then sum their partials through distributed shared memory, each
+// rank owning gn/S columns of the group.
+
+TG_HD int cl_begin(int r, int KB, int S) {
+    return static_cast<int>((static_cast<long long>(r) * KB) / S);
+}
+
+// The split S in {8, 4, 2, 1} for T groups of gn columns and KB k-units, or 0
+// (use stream-K): the largest S with no empty range (S <= KB), whole 32-column
+// warp slices per owner (gn a multiple of 32*S), T*S <= cap CTAs, and T*S at
+// least three quarters of num_sms (fewer CTAs would leave HBM bandwidth
+// unused).  `max_s` bounds S (a smaller maximum cluster on the device).
+inline int cl_split(long long T, long long KB, int gn, long long cap, int num_sms, int max_s) {
+    for (int S = 8; S >= 1; S >>= 1) {
+        if (S > max_s || S > KB || gn % (32 * S) != 0 || T * S > cap) continue;
+        return T * S * 4 >= 3ll * num_sms ? S : 0;
+    }
+    return 0;
+}
+
 // ------------------------------------------------------------ tile raster
 // Linear tile index t of an ntm x ntn tile grid -> (tm, tn).  Tiles are taken
 // in bands of group_m tile rows (the last band may be shorter); inside a band
