@@ -197,4 +197,48 @@ long long check_cl_split(long long* checked) {
     return bad;
 }
 
+// The CTA-pair kernel's hybrid schedule: the items cover every (tile,
+// k-block) exactly once; items past the whole tiles are the two halves of
+// the last R tiles (2R <= npairs, no half empty); handed out round-robin,
+// the halves of a tile go to two different pairs, each pair gets at most
+// one half and that is its last item.
+long long check_tail_schedule(long long* checked) {
+    long long bad = 0, n = 0;
+    for (int npairs = 1; npairs <= 80; ++npairs)
+    for (int tiles = 1; tiles <= 400; tiles += (tiles < 170 ? 1 : 7))
+    for (int kb = 1; kb <= 9; kb += 2) {
+        const int S = tg::tail_split(tiles, npairs, kb);
+        const int dp = tg::tail_dp(tiles, npairs, S);
+        const int items = tg::tail_items(tiles, dp, S);
+        const int R = tiles % npairs;
+        ++n; bad += !(S == 1 || S == 2);
+        ++n; bad += S == 2 && !(R > 0 && 2 * R <= npairs && kb >= 2 && dp == tiles - R);
+        ++n; bad += S == 1 && (dp != tiles || (R > 0 && 2 * R <= npairs && kb >= 2));
+        std::vector<int> cover(static_cast<size_t>(tiles) * kb, 0);
+        std::vector<int> last_item(npairs, -1), halves(npairs, 0), first_pair(tiles, -1);
+        for (int w = 0; w < items; ++w) {
+            int t, kb0, kb1, z;
+            tg::tail_item(w, dp, S, kb, t, kb0, kb1, z);
+            ++n;
+            if (t < 0 || t >= tiles || kb0 < 0 || kb1 > kb || kb0 >= kb1) { ++bad; continue; }
+            ++n; bad += (z >= 0) != (t >= dp);
+            for (int k = kb0; k < kb1; ++k) ++cover[static_cast<size_t>(t) * kb + k];
+            const int pr = w % npairs;
+            last_item[pr] = w;
+            if (z >= 0) {
+                ++halves[pr];
+                if (first_pair[t] < 0) first_pair[t] = pr;
+                else { ++n; bad += first_pair[t] == pr; }
+            }
+        }
+        for (int c : cover) { ++n; bad += c != 1; }
+        for (int pr = 0; pr < npairs; ++pr) {
+            ++n; bad += halves[pr] > 1;
+            if (halves[pr]) { ++n; bad += last_item[pr] < dp; }
+        }
+    }
+    *checked = n;
+    return bad;
+}
+
 }  // extern "C"

@@ -2,7 +2,9 @@
 
 The stream-K ranges of the weight-streaming kernels, their launch plan (how
 many split-K partial slots a column group needs), the split-K-in-a-cluster
-plan that replaces stream-K where it fills the GPU, the grouped raster of the
+plan that replaces stream-K where it fills the GPU, the CTA-pair kernel's
+hybrid schedule (whole tiles, then split halves of a thin last wave), the
+grouped raster of the
 persistent tile kernels and the fp32 split-K ranges are plain integer
 arithmetic shared by the device code and the launchers.  A wrong range here
 drops or double-counts part of the k sum, or leaves tiles unwritten, on some
@@ -34,7 +36,8 @@ def chk(tmp_path_factory):
                        ("check_sk_plan", []),
                        ("check_tile_coords", [ctypes.c_int, ctypes.c_int]),
                        ("check_ffma_splits", [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
-                       ("check_cl_split", [])):
+                       ("check_cl_split", []),
+                       ("check_tail_schedule", [])):
         fn = getattr(lib, name)
         fn.argtypes = args + [ctypes.POINTER(ll)]
         fn.restype = ll
@@ -75,4 +78,9 @@ def test_fp32_split_k_ranges(chk, num_sms):
 
 def test_cluster_split_plan(chk):
     bad, n = _run(chk.check_cl_split)
+    assert n > 100_000 and bad == 0
+
+
+def test_pair_kernel_tail_schedule(chk):
+    bad, n = _run(chk.check_tail_schedule)
     assert n > 100_000 and bad == 0

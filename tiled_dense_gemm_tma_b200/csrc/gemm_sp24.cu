@@ -317,7 +317,7 @@ int run_sp24(const GemmArgs& a, const void* E, int64_t lde, CUtensorMapDataType 
         return kCudaError;
     const long long tiles = ((a.M + SP::BM - 1) / SP::BM) * ((a.N + SP::BN - 1) / SP::BN);
     const int grid = static_cast<int>(persistent_grid(tiles, di->num_sms, a.ctas));
-    TcParams p;
+    TcParams p = {};
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);

@@ -60,6 +60,10 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     p.status = device_status_ptr();
     p.C = a.C;
     p.ldc = a.ldc;
+    p.tail_split = 1;
+    p.dp_tiles = 0;
+    p.tickets = nullptr;
+    p.ws = nullptr;
     if (!p.status) return kCudaError;
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(tA, tB, tC, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
@@ -91,6 +95,18 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
         return kCudaError;
     const long long tiles = ((a.M + Cfg::PM - 1) / Cfg::PM) * ((a.N + Cfg::BN - 1) / Cfg::BN);
     const int npairs = static_cast<int>(persistent_grid(tiles, di->num_sms / 2, a.ctas));
+    // hybrid schedule: the tiles of a thin last wave split in two along K,
+    // their halves meeting through the stream's workspace
+    const int num_kb = static_cast<int>((a.K + Cfg::BK - 1) / Cfg::BK);
+    const int S = tiles < 0x7fffffffll ? tail_split(static_cast<int>(tiles), npairs, num_kb) : 1;
+    const int dp = tail_dp(static_cast<int>(tiles), npairs, S);
+    int* tickets = nullptr;
+    float* ws = nullptr;
+    if (S > 1) {
+        const long long R = tiles - dp;
+        if (!stream_workspace(dev, a.stream, R * 4, R * 2 * Cfg::BM * Cfg::BN * 4, &tickets, &ws))
+            return kCudaError;
+    }
     TcParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
@@ -102,6 +118,10 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     p.status = device_status_ptr();
     p.C = a.C;
     p.ldc = a.ldc;
+    p.tail_split = S;
+    p.dp_tiles = dp;
+    p.tickets = tickets;
+    p.ws = ws;
     if (!p.status) return kCudaError;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * npairs, 1, 1);

@@ -80,6 +80,13 @@ struct TcParams {
     int* status;              // device status word (ST_TIMEOUT on an expired wait)
     void* C;                  // output base and row pitch (elements), for the ragged
     long long ldc;            // last column chunk, which is stored without TMA
+    // CTA-pair kernel only: hybrid schedule (tail_split / tail_dp of
+    // tile_sched.h) and, when split, its workspace: per tail tile and rank a
+    // check-in and a published word, and one 128 x 256 fp32 partial
+    int tail_split;
+    int dp_tiles;
+    int* tickets;
+    float* ws;
 };
 
 // Store the first `valid_bytes` (< 128) of one packed 128-byte output row

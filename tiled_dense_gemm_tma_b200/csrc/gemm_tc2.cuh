@@ -16,6 +16,17 @@
 //   empty[s]  in each CTA; the leader's MMA commit arrives on both.
 //   tfull[a]  in each CTA; the leader's MMA commit arrives on both.
 //   tempty[a] leader only; all 8 epilogue warps of the pair arrive (count 8).
+//
+// Hybrid schedule (tail_split / tail_item of tile_sched.h): whole tiles fill
+// the full waves; if the last wave holds at most half as many tiles as there
+// are pairs, each of those tiles is split into two halves of its k-blocks.
+// Per CTA (its 128 rows) the two halves meet through the workspace: each
+// checks in on a counter; the first writes its fp32 partial and publishes
+// it; the second waits for that, adds the partial into its accumulator in
+// TMEM and runs the ordinary epilogue (a + b is exact-order free: the two
+// possible orders give the same bits).  A half is the last item of its pair,
+// so its operand ring is idle by then: the partial goes out and comes in
+// through the ring by 128 KB bulk copies.
 // Loads are plain tiled TMA copies: each CTA reads only its own tiles into
 // its own shared memory.  Every wait is bounded; the CTAs meet on a cluster
 // barrier after set-up and before freeing TMEM.
@@ -52,6 +63,8 @@ struct Tc2Cfg {
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr int GROUP_M = 8;                   // pair-tile rows per raster band
     static constexpr int SMEM_DATA = STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * 2 * STG_BUF;
+    static constexpr int PART_BYTES = BM * BN * 4;      // one CTA's fp32 partial of a split tile
+    static_assert(STAGES * (A_STAGE + B_STAGE) >= PART_BYTES, "the ring holds a partial");
     static constexpr int SMEM_BYTES = SMEM_DATA + 256 + 1024;
 };
 
@@ -73,8 +86,12 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint64_t* tfull = empty + Cfg::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* epi_bar = drain + 1;             // this CTA's epilogue warps joined (count 4)
+    uint64_t* flag_bar = epi_bar + 1;          // check-in result published (count 1)
+    uint64_t* xbar = flag_bar + 1;             // a partner's partial landed in the ring
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* tail_flag = abort_flag + 1;      // [0] check-in result, [1] partner published
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -85,13 +102,21 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int ntn = (p.N + Cfg::BN - 1) / Cfg::BN;
     const int num_tiles = ntm * ntn;
     const int num_kb = (p.K + Cfg::BK - 1) / Cfg::BK;
+    const int S = p.tail_split > 1 ? p.tail_split : 1;
+    const int dp = S > 1 ? p.dp_tiles : num_tiles;
+    const int num_items = tail_items(num_tiles, dp, S);
     const uint64_t limit = p.timeout_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], 1); }
         for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 2 * Cfg::EPI_WARPS); }
         mbar_init(drain, 1);
+        mbar_init(epi_bar, Cfg::EPI_WARPS);
+        mbar_init(flag_bar, 1);
+        mbar_init(xbar, 1);
         *abort_flag = 0;
+        tail_flag[0] = 0;
+        tail_flag[1] = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -115,7 +140,9 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (elect_one()) {
             uint32_t armed = 0, armed_par = 0, it = 0;
             bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += npairs) {
+            for (int w = pair; w < num_items && ok; w += npairs) {
+                int t, kb0, kb1, z;
+                tail_item(w, dp, S, num_kb, t, kb0, kb1, z);
                 int tm, tn;
                 tile_coords(t, ntm, ntn, p.group_m, tm, tn);
                 const int m0 = tm * Cfg::PM + rank * Cfg::BM;
@@ -128,7 +155,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const uint32_t a_bytes = Cfg::A_MN ? a_live * Cfg::A_CHUNK : (a_live ? Cfg::A_STAGE : 0);
                 const uint32_t b_bytes = Cfg::B_MN ? b_live * Cfg::B_CHUNK : (b_live ? Cfg::B_STAGE : 0);
                 const uint32_t bytes = a_bytes + b_bytes;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
@@ -175,13 +202,15 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             constexpr uint32_t idesc = make_idesc(Cfg::FMT, Cfg::PM, Cfg::BN, Cfg::A_MN, Cfg::B_MN);
             uint32_t it = 0, tl = 0;
             bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += npairs, ++tl) {
+            for (int w = pair; w < num_items && ok; w += npairs, ++tl) {
+                int t, kb0, kb1, z;
+                tail_item(w, dp, S, num_kb, t, kb0, kb1, z);
                 const uint32_t acc = tl & 1;
                 const uint32_t aph = (tl >> 1) & 1;
                 if (!bounded_wait(&tempty[acc], aph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const uint32_t s = it % Cfg::STAGES;
                     const uint32_t ph = (it / Cfg::STAGES) & 1;
                     if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) { ok = false; break; }
@@ -198,7 +227,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const uint64_t bd = Cfg::B_MN
                             ? sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, 1024)
                             : sw128_desc(b_addr + k * 32, 16, 1024);
-                        mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+                        mma_f16_pair(d_tmem, ad, bd, idesc, (kb != kb0) || k != 0);
                     }
                     const uint32_t e_loc = smem_u32(&empty[s]);
                     mma_commit_pair(mapa_shared(e_loc, 0));      // both CTAs' slots
@@ -218,17 +247,124 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         // --------------------------------------------------- epilogue (both)
         const int q = warp & 3;
         uint8_t* stg0 = smStg + (warp - 2) * 2 * Cfg::STG_BUF;
-        uint32_t tl = 0, nstore = 0;
-        for (int t = pair; t < num_tiles; t += npairs, ++tl) {
+        uint32_t tl = 0, nstore = 0, nflag = 0, nepi = 0, nx = 0;
+        for (int w = pair; w < num_items; w += npairs, ++tl) {
+            int t, kb0, kb1, z;
+            tail_item(w, dp, S, num_kb, t, kb0, kb1, z);
             int tm, tn;
             tile_coords(t, ntm, ntn, p.group_m, tm, tn);
             const uint32_t acc = tl & 1;
             const uint32_t aph = (tl >> 1) & 1;
             if (!bounded_wait(&tfull[acc], aph, abort_flag, limit, p.status)) break;
             tc_fence_after();
-            epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
-                                                       tm * Cfg::PM + rank * Cfg::BM + q * 32,
-                                                       tn * Cfg::BN, stg0, nstore);
+            const int row0 = tm * Cfg::PM + rank * Cfg::BM + q * 32;
+            const uint32_t tmem_acc = tmem_base + acc * Cfg::BN + (static_cast<uint32_t>(q * 32) << 16);
+            bool store_tile = true;
+            if (z >= 0) {
+                // A half of a split tail tile.  One thread checks in and, as
+                // the second, waits for the partner's partial; each result
+                // reaches the other warps through flag_bar (one arrival per
+                // phase).  The first writes its partial, and the four warps
+                // meet on epi_bar before it is published.
+                int* ck = p.tickets + ((t - dp) * 2 + rank) * 2;     // [checked in, published]
+                // the CTA's 128 x 256 partial as [column / 4][row][4], the
+                // same in the workspace and in the ring: the 32 rows of a
+                // warp (one per lane) make each 16-byte access of the warp
+                // one contiguous 512-byte run of the ring
+                float* part = p.ws + static_cast<long long>((t - dp) * 2 + rank) * Cfg::BM * Cfg::BN;
+                float4* ring4 = reinterpret_cast<float4*>(smA) + q * 32 + lane;
+                if (warp == 2 && lane == 0) {
+                    *tail_flag = atomicAdd(ck, 1);
+                    mbar_arrive(flag_bar);
+                }
+                if (!bounded_wait(flag_bar, nflag & 1, abort_flag, limit, p.status)) break;
+                ++nflag;
+                const bool second = *tail_flag != 0;
+                if (!second) {
+                    fence_proxy_async_smem();          // copy engine and tensor core are done with the ring
+                    if (row0 < p.M) {
+#pragma unroll 1
+                        for (int c = 0; c < Cfg::BN; c += 32) {
+                            uint32_t v[32];
+                            tmem_ld_32x32b_x32(tmem_acc + c, v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                ring4[(c / 4 + j) * Cfg::BM] =
+                                    make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                        }
+                    }
+                    fence_proxy_async_smem();          // the ring's new contents, for the bulk store
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(epi_bar);
+                    if (!bounded_wait(epi_bar, nepi & 1, abort_flag, limit, p.status)) break;
+                    ++nepi;
+                    if (warp == 2 && lane == 0) {
+                        bulk_store_1d(part, smA, Cfg::PART_BYTES);
+                        bulk_commit();
+                        bulk_wait<0>();                 // written to global memory
+                        fence_proxy_async_global();
+                        __threadfence();
+                        atomicExch(ck + 1, 1);          // published
+                    }
+                    store_tile = false;
+                } else {
+                    // the partner checked in first: wait until it has published
+                    if (warp == 2 && lane == 0) {
+                        const uint64_t t0 = globaltimer_ns();
+                        int ok = 1;
+                        while (ld_acquire_gpu(ck + 1) == 0) {
+                            if (*abort_flag || globaltimer_ns() - t0 > limit) {
+                                *abort_flag = 1;
+                                atomicExch(p.status, ST_TIMEOUT);
+                                ok = 0;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                        if (ok) {
+                            atomicExch(ck, 0);                 // both words clean for the next call
+                            atomicExch(ck + 1, 0);
+                            fence_proxy_async_global();        // the partial, for the bulk load
+                            mbar_arrive_expect_tx(xbar, Cfg::PART_BYTES);
+                            bulk_load_1d(smA, part, Cfg::PART_BYTES, xbar);
+                        }
+                        tail_flag[1] = ok;
+                        mbar_arrive(flag_bar);
+                    }
+                    if (!bounded_wait(flag_bar, nflag & 1, abort_flag, limit, p.status)) break;
+                    ++nflag;
+                    if (!tail_flag[1]) break;
+                    if (!bounded_wait(xbar, nx & 1, abort_flag, limit, p.status)) break;
+                    ++nx;
+                    if (row0 < p.M) {
+                        // TMEM += partial, 32 columns at a time from the ring
+#pragma unroll 1
+                        for (int h = 0; h < Cfg::BN; h += 128) {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                uint32_t v[32];
+                                tmem_ld_32x32b_x32(tmem_acc + h + 32 * c, v);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const float4 a = ring4[(h / 4 + 8 * c + j) * Cfg::BM];
+                                    v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + a.x);
+                                    v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + a.y);
+                                    v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + a.z);
+                                    v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + a.w);
+                                }
+                                tmem_st_32x32b_x32(tmem_acc + h + 32 * c, v);
+                            }
+                        }
+                        tmem_st_wait();
+                    }
+                }
+            }
+            if (store_tile)
+                epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
+                                                           row0, tn * Cfg::BN, stg0, nstore);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));

@@ -277,7 +277,7 @@ int run_large(const GemmArgs& a) {
         return kCudaError;
     const long long tiles = ((a.M + W4::BM - 1) / W4::BM) * ((a.N + W4::BN - 1) / W4::BN);
     const int grid = static_cast<int>(persistent_grid(tiles, di->num_sms, a.ctas));
-    TcParams p;
+    TcParams p = {};
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);

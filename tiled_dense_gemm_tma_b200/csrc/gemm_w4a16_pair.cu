@@ -356,7 +356,7 @@ int run_pair(const GemmArgs& a) {
         return kCudaError;
     const long long tiles = ((a.M + W4P::PM - 1) / W4P::PM) * ((a.N + W4P::BN - 1) / W4P::BN);
     const int npairs = static_cast<int>(persistent_grid(tiles, di->num_sms / 2, a.ctas));
-    TcParams p;
+    TcParams p = {};
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);

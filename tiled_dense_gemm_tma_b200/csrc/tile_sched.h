@@ -98,6 +98,41 @@ inline int cl_split(long long T, long long KB, int gn, long long cap, int num_sm
     return 0;
 }
 
+// ------------------------------------------- hybrid schedule of the pairs
+// The persistent CTA-pair kernel hands out work items round-robin to its
+// npairs pairs.  Whole tiles fill the full waves; when the R tiles left for
+// the last wave would leave at least half of the pairs idle (2R <= npairs),
+// each of them is split into two halves of its k-blocks, so the last wave
+// takes about half a tile's time.  tail_dp() is the number of items that
+// are whole tiles (all tiles when there is no split).
+
+TG_HD int tail_split(int num_tiles, int npairs, int num_kb) {
+    const int R = num_tiles % npairs;
+    return (R > 0 && 2 * R <= npairs && num_kb >= 2) ? 2 : 1;
+}
+
+TG_HD int tail_dp(int num_tiles, int npairs, int S) {
+    return S > 1 ? num_tiles - num_tiles % npairs : num_tiles;
+}
+
+TG_HD int tail_items(int num_tiles, int dp, int S) { return dp + (num_tiles - dp) * S; }
+
+// Item w -> tile t, k-blocks [kb0, kb1), and the half z (-1 for a whole tile).
+TG_HD void tail_item(int w, int dp, int S, int num_kb, int& t, int& kb0, int& kb1, int& z) {
+    if (S <= 1 || w < dp) {
+        t = w;
+        kb0 = 0;
+        kb1 = num_kb;
+        z = -1;
+        return;
+    }
+    const int i = (w - dp) / S;
+    z = (w - dp) - i * S;
+    t = dp + i;
+    kb0 = static_cast<int>((static_cast<long long>(z) * num_kb) / S);
+    kb1 = static_cast<int>((static_cast<long long>(z + 1) * num_kb) / S);
+}
+
 // ------------------------------------------------------------ tile raster
 // Linear tile index t of an ntm x ntn tile grid -> (tm, tn).  Tiles are taken
 // in bands of group_m tile rows (the last band may be shorter); inside a band
