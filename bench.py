@@ -415,7 +415,11 @@ def flush_l2(bufs):
 
 
 def time_breakdown(case, iters, warmup, flush_buf):
-    """Median per-launch device time (s), flushing L2 before each launch."""
+    """Per-launch device time (s), flushing L2 before each launch: (median,
+    min, mean).  A launch's two event stamps land on a coarse grid on these
+    devices (steps of about 2 us at the end of short kernels), so the median
+    of a short kernel snaps to that grid; the mean over the launches, whose
+    phase against the grid varies, is the estimate the rates use."""
     import torch
     for _ in range(warmup):
         case.run()
@@ -430,7 +434,7 @@ def time_breakdown(case, iters, warmup, flush_buf):
         e.record()
         e.synchronize()
         ts.append(s.elapsed_time(e) * 1e-3)
-    return float(np.median(ts)), float(np.min(ts))
+    return float(np.median(ts)), float(np.min(ts)), float(np.mean(ts))
 
 
 def traffic_record(kernel_key):
@@ -589,7 +593,7 @@ def run_sweep(args):
     chosen, notes = [], []
     report = ["# Offline tile / stage sweep (tuning table)", "",
               "Command: `python bench.py --sweep` on one B200.  Each candidate is timed",
-              f"as the median of {args.breakdown_iters} launches per workload, L2 flushed "
+              f"as the mean of {args.breakdown_iters} launches per workload, L2 flushed "
               "before each launch; the default is the library's choice with no rule.  A class",
               f"takes a rule when its best candidate's geometric-mean time is more than "
               f"{SWEEP_MARGIN:.0%} below the default's.", ""]
@@ -603,7 +607,7 @@ def run_sweep(args):
             tg.tune_set([dict(base, **cand)] if cand else [])
             row = []
             for c in cases:
-                med, _ = time_breakdown(c, args.breakdown_iters, 3, flush)
+                _, _, med = time_breakdown(c, args.breakdown_iters, 3, flush)
                 if tg.last_device_status() != 0:
                     raise RuntimeError(f"device status after {op} {cand}")
                 row.append(med)
@@ -828,13 +832,14 @@ def main():
                 c = Case(name, dev, peaks)
                 c.run()
                 torch.cuda.synchronize()
-                med, mn = time_breakdown(c, args.breakdown_iters, 3, flush)
+                med, mn, mean = time_breakdown(c, args.breakdown_iters, 3, flush)
                 ok = tg.last_device_status() == 0
                 breakdown.append({"workload": name, "dtype": c.dtype,
-                                  "tflops": round(c.flops / med / 1e12, 2),
-                                  "gbs": round(c.alg_bytes / med / 1e9, 1),
+                                  "tflops": round(c.flops / mean / 1e12, 2),
+                                  "gbs": round(c.alg_bytes / mean / 1e9, 1),
+                                  "us_mean": round(mean * 1e6, 2),
                                   "us_median": round(med * 1e6, 2), "us_min": round(mn * 1e6, 2),
-                                  "bound": c.bound, "frac": round(c.achieved(med) / c.peak, 4),
+                                  "bound": c.bound, "frac": round(c.achieved(mean) / c.peak, 4),
                                   "peak": round(c.peak, 1), "peak_unit": c.unit,
                                   "status_ok": ok, "l2": "flushed (write + clean read of 512 MB) before each launch"})
                 del c
