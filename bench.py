@@ -416,10 +416,12 @@ def flush_l2(bufs):
 
 def time_breakdown(case, iters, warmup, flush_buf):
     """Per-launch device time (s), flushing L2 before each launch: (median,
-    min, mean).  A launch's two event stamps land on a coarse grid on these
-    devices (steps of about 2 us at the end of short kernels), so the median
-    of a short kernel snaps to that grid; the mean over the launches, whose
-    phase against the grid varies, is the estimate the rates use."""
+    min, trimmed mean).  A launch's two event stamps land on a coarse grid on
+    these devices (steps of about 2 us at the end of short kernels), so the
+    median of a short kernel snaps to that grid; the mean over the launches,
+    whose phase against the grid varies, does not.  The mean is taken over
+    the middle 80 % of the sorted times, so a rare slow launch (a clock dip,
+    another process) does not move it; it is the estimate the rates use."""
     import torch
     for _ in range(warmup):
         case.run()
@@ -434,7 +436,10 @@ def time_breakdown(case, iters, warmup, flush_buf):
         e.record()
         e.synchronize()
         ts.append(s.elapsed_time(e) * 1e-3)
-    return float(np.median(ts)), float(np.min(ts)), float(np.mean(ts))
+    srt = np.sort(np.asarray(ts))
+    cut = len(srt) // 10
+    mid = srt[cut:len(srt) - cut] if len(srt) > 2 * cut else srt
+    return float(np.median(srt)), float(srt[0]), float(np.mean(mid))
 
 
 def traffic_record(kernel_key):
@@ -593,7 +598,7 @@ def run_sweep(args):
     chosen, notes = [], []
     report = ["# Offline tile / stage sweep (tuning table)", "",
               "Command: `python bench.py --sweep` on one B200.  Each candidate is timed",
-              f"as the mean of {args.breakdown_iters} launches per workload, L2 flushed "
+              f"as the trimmed mean (middle 80 %) of {args.breakdown_iters} launches per workload, L2 flushed "
               "before each launch; the default is the library's choice with no rule.  A class",
               f"takes a rule when its best candidate's geometric-mean time is more than "
               f"{SWEEP_MARGIN:.0%} below the default's.", ""]
@@ -837,7 +842,7 @@ def main():
                 breakdown.append({"workload": name, "dtype": c.dtype,
                                   "tflops": round(c.flops / mean / 1e12, 2),
                                   "gbs": round(c.alg_bytes / mean / 1e9, 1),
-                                  "us_mean": round(mean * 1e6, 2),
+                                  "us_mean": round(mean * 1e6, 2),   # middle 80 % of the launches
                                   "us_median": round(med * 1e6, 2), "us_min": round(mn * 1e6, 2),
                                   "bound": c.bound, "frac": round(c.achieved(mean) / c.peak, 4),
                                   "peak": round(c.peak, 1), "peak_unit": c.unit,
