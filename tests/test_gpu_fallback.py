@@ -1,9 +1,9 @@
 """The one-CTA tensor-core kernels are the fallback when a cluster (CTA-pair)
 launch is refused.  TG_NO_PAIR=1 makes every pair launch report
 "unsupported" (read once per process, so the check runs in a child
-process); bf16, fp16, w4a16 and FP4-weight GEMMs with M > 128 must then still match the
-fp64 oracle at rtol = atol = 1e-2, on shapes with one tile per CTA and with
-more tiles than CTAs.
+process); bf16, fp16, w4a16 and FP4-weight GEMMs with M > 128, and the 2:4
+sparse GEMM, must then still match the fp64 oracle at rtol = atol = 1e-2, on
+shapes with one tile per CTA and with more tiles than CTAs.
 """
 import os
 import subprocess
@@ -48,6 +48,11 @@ CHILD = textwrap.dedent("""
         C = tg.gemm_wfp4(to_dev(A, "bf16"), to_dev(Bq, "u8"), to_dev(E, "u8"), N)
         assert_close(decode16(from_dev(C, "bf16"), "bf16"), oracle.gemm_wfp4(A, Bq, E, N=N),
                      1e-2, 1e-2, f"wfp4 {M}x{N}x{K}")
+    for (M, N, K) in ((300, 520, 200), (2048, 2600, 256)):
+        Ac, E, B, _ = synth.sp24(M, N, K, seed=2, dtype="bf16")
+        C = tg.gemm_sp24(to_dev(Ac, "bf16"), to_dev(E, "u8"), to_dev(B, "bf16"))
+        assert_close(decode16(from_dev(C, "bf16"), "bf16"), oracle.gemm_sp24(Ac, E, B, "bf16"),
+                     1e-2, 1e-2, f"sp24 {M}x{N}x{K}")
     torch.cuda.synchronize()
     print("RESULT", tg.last_device_status())
 """) % (ROOT, os.path.join(ROOT, "tests"))

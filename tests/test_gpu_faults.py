@@ -67,6 +67,13 @@ CHILD = textwrap.dedent("""
             call = lambda: tg.gemm_w4a16(dA, dB, dS, N)
             conv = lambda C: decode16(from_dev(C, "f16"), "f16")
             tol = (1e-2, 1e-2)
+        elif fam.startswith("sp24"):
+            Ac, E, B, _ = synth.sp24(512, 768, 1024, seed=2, dtype="bf16")
+            dA, dE, dB = to_dev(Ac, "bf16"), to_dev(E, "u8"), to_dev(B, "bf16")
+            ref = oracle.gemm_sp24(Ac, E, B, "bf16")
+            call = lambda: tg.gemm_sp24(dA, dE, dB)
+            conv = lambda C: decode16(from_dev(C, "bf16"), "bf16")
+            tol = (1e-2, 1e-2)
         else:
             M, N, K = {"wfp4_pair": (512, 1024, 1024), "wfp4_large": (512, 1024, 1024),
                        "skinny_wfp4": (16, 2048, 4096)}[fam]
@@ -100,8 +107,9 @@ CHILD = textwrap.dedent("""
 
 FAMILIES = ["tc2_bf16", "tf32", "skinny_bf16", "skinny_bf16_tb", "gemv_bf16", "ffma",
             "ffma_splitk", "w4a16_pair", "skinny_w4a16", "gemv_w4a16", "wfp4_pair",
-            "skinny_wfp4", "tc_bf16", "w4a16_large", "wfp4_large"]
-ONE_CTA = {"tc_bf16", "w4a16_large", "wfp4_large"}      # run with the CTA-pair kernels off
+            "skinny_wfp4", "sp24_pair", "tc_bf16", "w4a16_large", "wfp4_large", "sp24_one"]
+# run with the CTA-pair kernels off
+ONE_CTA = {"tc_bf16", "w4a16_large", "wfp4_large", "sp24_one"}
 
 
 @pytest.mark.parametrize("family", FAMILIES)

@@ -58,7 +58,7 @@ int* device_status_ptr();
 //   16-27  gemm_skinny.cu    28-35  gemm_skinny.cu (weights stored transposed)
 //   36-39  gemm_skinny.cu (FP4 weights)
 //   40-48  gemv.cu           50-53  gemm_skinny_static.cu
-//   56-57  gemm_sp24.cu
+//   56-57  gemm_sp24.cu (one CTA)   61-62  gemm_sp24.cu (CTA pairs)
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 
 // Clusters of S CTAs (threads and dynamic shared memory bytes each) of the

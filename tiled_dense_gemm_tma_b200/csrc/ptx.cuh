@@ -466,6 +466,19 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
+// The sparse form on CTA pairs: A (both CTAs' shared memory, compressed,
+// M split) with each CTA's position codes in its own tensor memory at the
+// same address e_tmem.
+__device__ __forceinline__ void mma_f16_sp_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate, uint32_t e_tmem) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+        : "memory");
+}
+
 // Arrive once on the mbarrier at shared::cluster address `bar_cl` (this CTA
 // or the peer) when this thread's prior tcgen05 ops of the pair complete.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar_cl) {
