@@ -609,7 +609,10 @@ def run_sweep(args):
         allc = [{}] + list(cands)
         times = []
         for cand in allc:
-            tg.tune_set([dict(base, **cand)] if cand else [])
+            # the default too runs under a rule of the class, with every field
+            # at its default: it masks the built-in rules, which a sweep must
+            # not take as the default it measures against
+            tg.tune_set([dict(base, **cand)])
             row = []
             for c in cases:
                 _, _, med = time_breakdown(c, args.breakdown_iters, 3, flush)

@@ -7,9 +7,9 @@
 namespace tg {
 
 constexpr TuneRule kBuiltinRules[] = {
-    {0, 2, 5, 64, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // bf16 M 5..64: path=small_m, ctas=128 (0.937 of the default)
-    {0, 3, 65, 128, 4096, 0x7fffffffffffffffll, 0, 0, 0, 0},   // bf16 M 65..128: path=cta_pair (0.846 of the default)
-    {2, 1, 1, 4, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 1..4: path=cuda_core, ctas=128 (0.924 of the default)
+    {0, 3, 65, 128, 4096, 0x7fffffffffffffffll, 0, 0, 0, 0},   // bf16 M 65..128: path=cta_pair (0.879 of the default)
+    {2, 1, 1, 4, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 1..4: path=cuda_core, ctas=128 (0.938 of the default)
+    {2, 2, 5, 128, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 5..128: path=small_m, ctas=128 (0.978 of the default)
     {-1, 0, 0, 0, 0, 0, 0, 0, 0, 0},   // end: matches nothing
 };
 
