@@ -148,6 +148,20 @@ __device__ __forceinline__ uint32_t bf16_pow2_pair(uint32_t t) { return t << 7; 
 // skipped; f2 is then left unset.  A NaN scale (E = 255) makes f2 NaN.
 __device__ __forceinline__ bool fp4_scale_pairs(uint32_t e_lo, uint32_t e_hi, uint32_t (&f1)[4],
                                                 uint32_t (&f2)[4]) {
+    // Every E <= 128 (the usual case): m1 = E + 126 byte by byte and m2 = 1,
+    // the same factors as the general path below at a fraction of its
+    // per-byte min / max / compare work.  A byte is above 128 exactly when
+    // its bit 7 is set and some lower bit too.
+    const uint32_t above = (((e_lo & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) & e_lo) |
+                           (((e_hi & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) & e_hi);
+    if ((above & 0x80808080u) == 0) {
+        const uint32_t a = e_lo + 0x7E7E7E7Eu, b = e_hi + 0x7E7E7E7Eu;   // <= 254: no carries
+        f1[0] = bf16_pow2_pair(__byte_perm(a, 0u, 0x4240));
+        f1[1] = bf16_pow2_pair(__byte_perm(b, 0u, 0x4240));
+        f1[2] = bf16_pow2_pair(__byte_perm(a, 0u, 0x4341));
+        f1[3] = bf16_pow2_pair(__byte_perm(b, 0u, 0x4341));
+        return false;
+    }
     uint32_t a1, a2, b1, b2;
     e8m0_factor_bytes(e_lo, a1, a2);
     e8m0_factor_bytes(e_hi, b1, b2);
