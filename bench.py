@@ -615,7 +615,7 @@ def run_sweep(args):
             tg.tune_set([dict(base, **cand)])
             row = []
             for c in cases:
-                _, _, med = time_breakdown(c, args.breakdown_iters, 3, flush)
+                _, _, med = time_breakdown(c, args.breakdown_iters, 10, flush)
                 if tg.last_device_status() != 0:
                     raise RuntimeError(f"device status after {op} {cand}")
                 row.append(med)
@@ -664,7 +664,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--breakdown-iters", type=int, default=30)
+    ap.add_argument("--breakdown-iters", type=int, default=50)
     ap.add_argument("--sweep", action="store_true",
                     help="time the tuning table's candidates and rewrite its built-in rules")
     return ap.parse_args()
@@ -872,7 +872,7 @@ def main():
                 c = Case(name, dev, peaks)
                 c.run()
                 torch.cuda.synchronize()
-                med, mn, mean = time_breakdown(c, args.breakdown_iters, 3, flush)
+                med, mn, mean = time_breakdown(c, args.breakdown_iters, 10, flush)
                 ok = tg.last_device_status() == 0
                 breakdown.append({"workload": name, "dtype": c.dtype,
                                   "tflops": round(c.flops / mean / 1e12, 2),
