@@ -38,8 +38,11 @@
  *   the life of the process, a small status word (see
  *   tg_last_device_status), a cache of tensor-copy descriptors, and one
  *   split-K workspace per (device, stream): fp32 partials and tile tickets
- *   of the kernels that split K across CTAs (M <= 128, and fp32 shapes with
- *   fewer 128 x 128 tiles than SMs).  It is allocated on the first such call
+ *   of the kernels that split K across CTAs through global memory (small M
+ *   where the split does not run inside thread-block clusters, fp32 shapes
+ *   with fewer 128 x 128 tiles than SMs, and 16-bit GEMMs with M > 128 whose
+ *   last wave of 256 x 256 tiles is split along K).  It is allocated on the
+ *   first such call
  *   on a stream (at least 8 MiB), grown when a larger call needs it (the
  *   regrow frees the old one, which synchronises the device), and reused.
  *   Calls on one stream share it; calls on different streams get their own
@@ -249,14 +252,17 @@ TG_API tg_status tg_gemm_sp24_bf16(int64_t M, int64_t N, int64_t K,
  *
  * Same arguments, semantics and alignment rules as tg_gemm_bf16; M must be
  * <= 128 (else TG_ERR_UNSUPPORTED).  It always runs the small-M tensor-core
- * kernel (tg_gemm_bf16 takes a CUDA-core kernel for M <= 4).  The split-K
- * scratch of that kernel lives in a fixed device array of 16 MiB of fp32 partials plus 4096
+ * kernel (tg_gemm_bf16 takes a CUDA-core kernel for M <= 4), with the same
+ * plan as tg_gemm_bf16 on all SMs.  Shapes whose split-K runs inside
+ * thread-block clusters need no scratch.  For the others the split-K
+ * scratch lives in a fixed device array of 16 MiB of fp32 partials plus 4096
  * tile tickets that is part of the library image; shapes needing more return
  * TG_ERR_UNSUPPORTED.  Every call shares that array (tickets are cleared at
  * the start of each call): calls that overlap on the GPU, e.g. on two
  * streams, race and give wrong results -- serialise them.  The first call on
  * each device looks up the array's device address (cudaGetSymbolAddress) and
- * caches it; make that first call before any stream capture.
+ * how many clusters of the kernel the device holds at once, and caches both;
+ * make that first call before any stream capture.
  */
 TG_API tg_status tg_gemm_bf16_small_m_static(int64_t M, int64_t N, int64_t K,
                                              const void *A, int64_t lda,
