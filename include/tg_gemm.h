@@ -46,10 +46,12 @@
  *   on a stream (at least 8 MiB), grown when a larger call needs it (the
  *   regrow frees the old one, which synchronises the device), and reused.
  *   Calls on one stream share it; calls on different streams get their own
- *   (cudaStreamPerThread counts as one stream per host thread).  To capture
- *   such calls into a CUDA graph, make one uncaptured call of the largest
- *   shape on that stream first: a capture cannot allocate.
- *   tg_gemm_bf16_small_m_static avoids it.
+ *   (cudaStreamPerThread counts as one stream per host thread).  A stream
+ *   under CUDA graph capture never allocates it: there the 16-bit GEMM with
+ *   M > 128 runs its last wave of tiles whole, and the other users of the
+ *   workspace return TG_ERR_CUDA unless one uncaptured call of the largest
+ *   shape on that stream came first.  tg_gemm_bf16_small_m_static avoids
+ *   it.
  * - Thread safety: calls from several host threads are allowed.  A thread
  *   needs no earlier CUDA call: on its first call the library makes the
  *   current device's primary context current on that thread.

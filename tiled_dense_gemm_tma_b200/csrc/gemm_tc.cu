@@ -98,14 +98,21 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     // hybrid schedule: the tiles of a thin last wave split in two along K,
     // their halves meeting through the stream's workspace
     const int num_kb = static_cast<int>((a.K + Cfg::BK - 1) / Cfg::BK);
-    const int S = tiles < 0x7fffffffll ? tail_split(static_cast<int>(tiles), npairs, num_kb) : 1;
-    const int dp = tail_dp(static_cast<int>(tiles), npairs, S);
+    int S = tiles < 0x7fffffffll ? tail_split(static_cast<int>(tiles), npairs, num_kb) : 1;
+    int dp = tail_dp(static_cast<int>(tiles), npairs, S);
     int* tickets = nullptr;
     float* ws = nullptr;
     if (S > 1) {
         const long long R = tiles - dp;
-        if (!stream_workspace(dev, a.stream, R * 4, R * 2 * Cfg::BM * Cfg::BN * 4, &tickets, &ws))
-            return kCudaError;
+        if (!stream_workspace(dev, a.stream, R * 4, R * 2 * Cfg::BM * Cfg::BN * 4, &tickets, &ws)) {
+            // no workspace (a stream under graph capture that has none yet,
+            // or no memory): the last wave runs whole tiles
+            cudaGetLastError();
+            S = 1;
+            dp = static_cast<int>(tiles);
+            tickets = nullptr;
+            ws = nullptr;
+        }
     }
     TcParams p;
     p.M = static_cast<int>(a.M);

@@ -1,6 +1,7 @@
 // workspace.cu -- per-(device, stream) scratch of the kernels that split K
-// across CTAs (the small-M tensor-core kernel, the M <= 4 CUDA-core kernel
-// and the fp32 FFMA kernel when tiles are fewer than SMs).
+// across CTAs through global memory (the small-M tensor-core kernel's
+// stream-K, the M <= 4 CUDA-core kernel, the fp32 FFMA kernel when tiles are
+// fewer than SMs, and the CTA-pair kernel's split last wave).
 #include "launch.h"
 
 #include <cuda_runtime.h>
@@ -46,6 +47,12 @@ bool stream_workspace(int dev, void* stream, long long tickets, long long partia
     std::lock_guard<std::mutex> lk(g_ws_mu);
     Workspace& w = g_ws[ws_key(dev, stream)];
     if (!w.base || w.ticket_cap < tickets || w.partial_cap < partial_bytes) {
+        // a stream being captured into a graph cannot allocate (and a failed
+        // allocation there would invalidate the capture): report "none"
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess ||
+            cs != cudaStreamCaptureStatusNone)
+            return false;
         if (w.base) {
             cudaFree(w.base);     // synchronises the device: no kernel still uses it
             w.base = nullptr;
