@@ -17,9 +17,10 @@
 //   warp w takes a run of consecutive rows (vector reads fetch their
 //   activations); each lane its GN/32
 //   neighbouring columns of a row.  16-bit weights widen exactly to fp32 and
-//   multiply into fp32 accumulators.  Signed 4-bit weights decode exactly
-//   (nib_frac), and per unit a lane forms sum_k q[k][n] a[k] exactly-rounded
-//   in fp32, which the group scale s[g][n] multiplies once per unit (the
+//   multiply into fp32 accumulators.  Signed 4-bit weights decode exactly,
+//   two per logic op, into fp16 pairs (nib_pair); mixed-precision FMAs (fp16
+//   inputs, fp32 accumulator) form per unit and lane sum_k q[k][n] a[k] in
+//   fp32, which the group scale s[g][n] multiplies once per unit (the
 //   dequantised weight W = q * s of the pages' dequantize GEMM, with the
 //   scale factored out of the unit's sum).
 // * At a segment's end the warps' sums are added in warp order through
@@ -80,31 +81,33 @@ struct GvCfg {
 };
 
 
-// Paired fp32 arithmetic (two independent IEEE operations per instruction,
-// each rounded as its scalar form).
-__device__ __forceinline__ uint64_t pk(float x, float y) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+// Exact decode of signed 4-bit weights to fp16 pairs, two weights per
+// logic op and without a subtraction per weight.  With b = q + 8 in [0, 15]
+// (the nibble with bit 3 flipped) placed at mantissa bit p of an fp16 1.0,
+// the half is f = 1 + b / D with D = 2^(10 - p); f has at most 11
+// significant bits, so f * a is exact in fp32 for an fp16 activation a, and
+//     sum_k q[k] a[k] = D sum_k f[k] a[k] - (D + 8) sum_k a[k].
+// One lop3 keeps the nibbles at bits p and p + 16 of x, flips their bit 3
+// and sets the exponent of 1.0 in both halves: per bit, lanes of `keep`
+// take x (xor the flip bit of `set`), the rest take `set`.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t x, uint32_t keep, uint32_t set) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(x), "r"(keep), "r"(set));
     return r;
 }
-__device__ __forceinline__ float2 upk(uint64_t v) {
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-    return r;
-}
-__device__ __forceinline__ void fma2(uint64_t& d, uint64_t x, uint64_t y) {
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(x), "l"(y));
-}
+constexpr uint32_t kKeepLo = 0x000F000Fu, kSetLo = 0x3C083C08u;   // nibbles at bits 0, 16: D = 1024
+constexpr uint32_t kKeepHi = 0x00F000F0u, kSetHi = 0x3C803C80u;   // nibbles at bits 4, 20: D = 64
 
-// Exact decode of signed 4-bit weights to fp32 without a subtraction per
-// weight: with b = q + 8 in [0, 15] (the nibble with bit 3 flipped), the
-// float f = 1 + b / 16 is built by placing b under the exponent of 1.0
-// (bits 0x3F800000 | b << 19); f * a is exact for an fp16 activation a
-// (5 x 11 significant bits), and q = 16 f - 24, so
-//     sum_k q[k] a[k] = 16 sum_k f[k] a[k] - 24 sum_k a[k].
-// `t3` holds (b << 3) | 0x80 in each byte; byte i gives f.
-__device__ __forceinline__ float nib_frac(uint32_t t3, int i) {
-    return __uint_as_float(__byte_perm(t3, 0x3Fu, 0x4055u | (static_cast<uint32_t>(i) << 8)));
+// The two halves of a packed fp16 pair, and fp32 += fp16 x fp16 (one
+// rounding; the product of two fp16 values is exact in fp32).
+__device__ __forceinline__ void halves(uint32_t v, unsigned short& lo, unsigned short& hi) {
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
+}
+__device__ __forceinline__ void fma_f16_f32(float& d, unsigned short x, unsigned short y) {
+    asm("fma.rn.f32.f16 %0, %1, %2, %0;" : "+f"(d) : "h"(x), "h"(y));
+}
+__device__ __forceinline__ void add_f16_f32(float& d, unsigned short x) {
+    asm("add.rn.f32.f16 %0, %1, %0;" : "+f"(d) : "h"(x));
 }
 
 // Two activations (or 16-bit weights) packed in a word, widened to fp32.
@@ -247,13 +250,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 return (i & 1) ? f.y : f.x;
             };
             if constexpr (Cfg::Q4) {
-                uint64_t facc[MR][CPL / 2];                  // column pairs
+                // f sums per column (nibble j of the lane's word is column j)
+                float fac[MR][CPL];
                 float suma[MR];
 #pragma unroll
                 for (int m = 0; m < MR; ++m) {
                     suma[m] = 0.f;
 #pragma unroll
-                    for (int q = 0; q < CPL / 2; ++q) facc[m][q] = 0ull;
+                    for (int q = 0; q < CPL; ++q) fac[m][q] = 0.f;
                 }
 #pragma unroll
                 for (int i = 0; i < RPW; ++i) {
@@ -262,22 +266,23 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                     // unit lane / 4, stored at unit (lane / 4) ^ (r % 8))
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(
                         slot + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
-                    const uint32_t tq = w ^ 0x88888888u;                          // b = q + 8
-                    const uint32_t te = ((tq << 3) & 0x78787878u) | 0x80808080u;  // columns 0, 2, 4, 6
-                    const uint32_t to = ((tq >> 1) & 0x78787878u) | 0x80808080u;  // columns 1, 3, 5, 7
-                    uint64_t a2[MR];                                               // (a, a)
+                    const uint32_t w8 = w >> 8;
+                    // pair j holds columns (j, j + 4): D = 1024 for even j, 64 for odd j
+                    const uint32_t hp[4] = {nib_pair(w, kKeepLo, kSetLo), nib_pair(w, kKeepHi, kSetHi),
+                                            nib_pair(w8, kKeepLo, kSetLo), nib_pair(w8, kKeepHi, kSetHi)};
 #pragma unroll
                     for (int m = 0; m < MR; ++m) {
-                        const float am = act(m, i);
-                        a2[m] = pk(am, am);
-                        suma[m] += am;
-                    }
+                        unsigned short a_lo, a_hi;
+                        halves(avw[m][i >> 1], a_lo, a_hi);
+                        const unsigned short am = (i & 1) ? a_hi : a_lo;
+                        add_f16_f32(suma[m], am);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        // columns (2 j, 2 j + 1) as one pair
-                        const uint64_t f2 = pk(nib_frac(te, j), nib_frac(to, j));
-#pragma unroll
-                        for (int m = 0; m < MR; ++m) fma2(facc[m][j], f2, a2[m]);
+                        for (int j = 0; j < 4; ++j) {
+                            unsigned short lo, hi;
+                            halves(hp[j], lo, hi);
+                            fma_f16_f32(fac[m][j], lo, am);
+                            fma_f16_f32(fac[m][j + 4], hi, am);
+                        }
                     }
                 }
                 // the unit's rows share one scale group: total += s * sum_k q a
@@ -292,12 +297,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 }
 #pragma unroll
                 for (int m = 0; m < MR; ++m) {
-                    const float nb = -24.f * suma[m];
 #pragma unroll
-                    for (int j = 0; j < CPL / 2; ++j) {
-                        const float2 f = upk(facc[m][j]);
-                        acc[m][2 * j] = fmaf(sc[2 * j], fmaf(16.f, f.x, nb), acc[m][2 * j]);
-                        acc[m][2 * j + 1] = fmaf(sc[2 * j + 1], fmaf(16.f, f.y, nb), acc[m][2 * j + 1]);
+                    for (int j = 0; j < CPL; ++j) {
+                        const float d = (j & 1) ? 64.f : 1024.f;
+                        acc[m][j] = fmaf(sc[j], fmaf(d, fac[m][j], -(d + 8.f) * suma[m]), acc[m][j]);
                     }
                 }
             } else {
