@@ -135,10 +135,13 @@ TG_API tg_status tg_gemm_bf16(int64_t M, int64_t N, int64_t K,
  *   trans_b = 0: B is K x N, row pitch ldb >= N;  trans_b = 1: B is stored
  *                N x K (op(B) = B^T), row pitch ldb >= K.
  * trans flags other than 0 / 1 -> TG_ERR_INVALID_ARG.  With both flags 0
- * this is tg_gemm_f16 / tg_gemm_bf16.  A call with only B transposed and
- * M <= 128 runs the weight-streaming small-M kernel on K-major weight
- * tiles; every other transposed call runs the CTA-pair tensor-core kernel
- * and returns TG_ERR_UNSUPPORTED if the device refuses its cluster launch.
+ * this is tg_gemm_f16 / tg_gemm_bf16.  A call with only B transposed takes
+ * the kernel family that the plain call's tuning rule (tg_tune_rule, op
+ * TG_OP_F16 / TG_OP_BF16) picks for its M and N: with M <= 128 and the
+ * small-M or CUDA-core path, the weight-streaming small-M kernel on K-major
+ * weight tiles; otherwise the CTA-pair kernel.  Every other transposed call
+ * runs the CTA-pair tensor-core kernel.  A refused cluster launch of the
+ * CTA-pair kernel returns TG_ERR_UNSUPPORTED.
  * Same alignment, status and ownership rules as tg_gemm_f16.
  */
 TG_API tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K,

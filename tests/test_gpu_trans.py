@@ -7,7 +7,8 @@ stored transposes.  Tolerance rtol = atol = 1e-2 as for the plain 16-bit
 GEMM; integer data in {-1, 0, 1} must match bit-exactly.  Shapes include
 ragged edges in every dimension, M below the 256-row pair tile, more pair
 tiles than CTA pairs, and small M with B transposed (the weight-streaming
-kernel on K-major weight tiles).
+kernel on K-major weight tiles, or the CTA-pair kernel where the tuning rule
+picks it).
 """
 import numpy as np
 import pytest
@@ -147,3 +148,21 @@ def test_matmul_backward(tg, kind):
     assert_close(got_dB, ref_dB, RTOL, ATOL, "dB")
     assert rel_frob(got_dA, ref_dA) <= FROB[kind]
     assert rel_frob(got_dB, ref_dB) <= FROB[kind]
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f16"])
+@pytest.mark.parametrize("path", ["small_m", "cta_pair"])
+@pytest.mark.parametrize("shape", [(128, 14336, 4096), (100, 777, 1200), (3, 1000, 700)])
+def test_small_m_transposed_b_follows_tuning_rule(tg, kind, path, shape):
+    # A B-transposed call takes the plain call's rule: each forced kernel
+    # family gives the oracle's result, ragged shapes included
+    M, N, K = shape
+    A, B = synth.normal(M, N, K, seed=4, dtype=kind, scale_by_sqrt_k=True)
+    ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B)
+    tg.tune_set([{"op": kind, "path": path, "m_lo": 1, "m_hi": 128}])
+    try:
+        got = decode16(_run(tg, kind, A, B, False, True), kind)
+    finally:
+        tg.tune_set([])
+    assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} {path}")
+    assert rel_frob(got, ref) <= FROB[kind]

@@ -127,7 +127,7 @@ tg_status tg_gemm_f16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_t
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
     tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
-    if (!trans_a && !trans_b) a = tg::with_rule(a, tg::tune_lookup(tg::OP_F16, M, N));
+    if (!trans_a) a = tg::with_rule(a, tg::tune_lookup(tg::OP_F16, M, N));
     return static_cast<tg_status>(tg::launch_tc_trans(a, 0, trans_a, trans_b));
 }
 
@@ -138,7 +138,7 @@ tg_status tg_gemm_bf16_ex(int64_t M, int64_t N, int64_t K, const void* A, int64_
     if (s != TG_OK || M == 0 || N == 0) return s;
     if (K == 0) return zero_fill(C, ldc, M, N, 2, stream);
     tg::GemmArgs a = make_args(M, N, K, A, lda, B, ldb, C, ldc, epilogue, stream);
-    if (!trans_a && !trans_b) a = tg::with_rule(a, tg::tune_lookup(tg::OP_BF16, M, N));
+    if (!trans_a) a = tg::with_rule(a, tg::tune_lookup(tg::OP_BF16, M, N));
     return static_cast<tg_status>(tg::launch_tc_trans(a, 1, trans_a, trans_b));
 }
 

@@ -181,14 +181,16 @@ int launch_tc_f16(const GemmArgs& a) {
     }
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
 }
-// 16-bit GEMM with optionally transposed operands.  Only B transposed with
-// M <= 128 (the backward product dA = dC . B^T at small batch) runs the
-// weight-streaming kernel on K-major weight tiles; every other transposed
-// call runs the CTA-pair kernel (no one-CTA variant: a refused cluster
-// launch reports kUnsupported).
+// 16-bit GEMM with optionally transposed operands.  Only B transposed (the
+// backward product dA = dC . B^T) follows the plain call's path choice: with
+// M <= 128 and the small-M or CUDA-core path it runs the weight-streaming
+// kernel on K-major weight tiles (there is no transposed CUDA-core kernel).
+// Every other transposed call runs the CTA-pair kernel (no one-CTA variant:
+// a refused cluster launch reports kUnsupported).
 int launch_tc_trans(const GemmArgs& a, int bf16, int trans_a, int trans_b) {
     if (!trans_a && !trans_b) return bf16 ? launch_tc_bf16(a) : launch_tc_f16(a);
-    if (!trans_a && a.M <= kSkinnyMaxM) return launch_skinny_trans_b(a, bf16);
+    if (!trans_a && a.M <= kSkinnyMaxM && a.path != PATH_CTA_PAIR && a.path != PATH_ONE_CTA)
+        return launch_skinny_trans_b(a, bf16);
     const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (bf16) {
         if (trans_a && trans_b) return run_pair<Cfg2T11<1, OutT::BF16>>(a, dt, 11);
