@@ -4,7 +4,8 @@ bf16, fp16 and 4-bit weights) against the fp64 oracle, through the C ABI.
 Shapes cover ragged column tails (N not a multiple of the 256 or 512
 columns a CTA owns, odd N for packed weights), ragged K (not a multiple of
 the 128-row groups), K long enough to be split over several CTAs (partials
-summed by the last CTA of a column block), ReLU, and the bit-exact cases:
+summed in a cluster through distributed shared memory, or by the last CTA
+of a column block under stream-K), ReLU, and the bit-exact cases:
 integer data in {-1, 0, 1} (16-bit weights) and power-of-two scales with
 integer activations (4-bit weights).  Repeated calls must agree bit for bit
 (the split-K partials are summed in a fixed order).
@@ -113,3 +114,41 @@ def test_gemv_w4a16_bit_exact_groups_and_repeatable(tg):
     first = _run4(tg, A, Bq, S, 8192)
     for _ in range(3):
         assert np.array_equal(_run4(tg, A, Bq, S, 8192), first)
+
+
+CLUSTER_SHAPES = [(1, 8000, 1280), (3, 8192, 640), (4, 4000, 1024), (2, 8192, 8192)]
+
+
+@pytest.mark.parametrize("kind", ["w4a16", "bf16", "f16"])
+@pytest.mark.parametrize("shape", CLUSTER_SHAPES)
+def test_gemv_cluster_and_stream_k_splits(tg, kind, shape):
+    # These shapes give T column groups x a split S of 2 to 8 that fill the
+    # GPU, so by default a group's k-range is split inside a cluster and the
+    # partials meet in distributed shared memory (ragged N, a k-range of 5
+    # units over 4 ranks, ragged K for 16-bit weights).  Capping the grid at
+    # 100 CTAs leaves no such split and forces stream-K.  Both match the
+    # oracle; each is repeatable bit for bit.
+    M, N, K = shape
+    if kind == "w4a16":
+        A, Bq, S, _ = synth.w4a16(M, N, K, seed=5)
+        ref = oracle.gemm_w4a16(A, Bq, S, N=N, relu=True)
+        run = lambda: _run4(tg, A, Bq, S, N, relu=True)
+        frob = 2e-3
+    else:
+        K = K - 24                                   # ragged in K
+        A, B = synth.normal(M, N, K, seed=5, dtype=kind, scale_by_sqrt_k=True)
+        ref = (oracle.gemm_bf16 if kind == "bf16" else oracle.gemm_f16)(A, B, True)
+        run = lambda: _run16(tg, kind, A, B, relu=True)
+        frob = FROB[kind]
+    for ctas in (0, 100):
+        if ctas:
+            tg.tune_set([{"op": kind, "path": "cuda_core", "m_lo": 1, "m_hi": 4, "ctas": ctas}])
+        try:
+            first = run()
+            again = run()
+        finally:
+            tg.tune_set([])
+        assert np.array_equal(first, again)
+        got = decode16(first, "f16" if kind == "w4a16" else kind)
+        assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} ctas={ctas}")
+        assert rel_frob(got, ref) <= frob

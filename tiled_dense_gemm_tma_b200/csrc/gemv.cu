@@ -6,10 +6,12 @@
 // rows, and the 4-bit weights would have to be written back to shared memory
 // as fp16 for it.  Here the weights are multiplied where they land:
 //
-// * Stream-K split as in the weight-streaming tensor-core kernel: the units
-//   (GN columns x BK rows of weights) of all column groups are cut into one
-//   contiguous, equal range per SM; a maximal run of a range inside one
-//   column group is a segment.
+// * The k-split of the weight-streaming tensor-core kernel.  Where T column
+//   groups (GN columns each) times a split S of 2 to 8 fill the GPU, group t
+//   goes to the S CTAs of cluster t, each taking a contiguous part of its
+//   units (GN columns x BK rows of weights).  Otherwise stream-K: the units
+//   of all groups are cut into one contiguous, equal range per SM; a maximal
+//   run of a range inside one column group is a segment.
 // * Warp 0 streams each unit by TMA into a ring of shared-memory slots: the
 //   weight tile (128-byte swizzled rows), for 4-bit weights the unit's fp16
 //   scale row, and the activations (MR rows x 64 values per slice).
@@ -24,10 +26,14 @@
 //   dequantised weight W = q * s of the pages' dequantize GEMM, with the
 //   scale factored out of the unit's sum).
 // * At a segment's end the warps' sums are added in warp order through
-//   shared memory.  A segment that covers its whole column group writes C;
-//   otherwise the fp32 partial goes to a fixed workspace slot (row-major)
-//   and the CTA that takes the group's last ticket adds the slots in segment
-//   order -- deterministic -- applies ReLU, rounds and writes C.
+//   shared memory.  A segment that covers its whole column group writes C.
+//   In a cluster, rank o owns GN/S columns of the group: every rank stores
+//   its partial of them into rank o's receive buffer (distributed shared
+//   memory) and rank o adds the partials in rank order.  Under stream-K the
+//   fp32 partial goes to a fixed workspace slot (row-major) and the CTA that
+//   takes the group's last ticket adds the slots in segment order.  Both
+//   orders are fixed (deterministic); the last adder applies ReLU, rounds
+//   and writes C.
 // Every wait is bounded (mbarriers, timeout -> device status 5).
 #include "gemm_skinny.cuh"   // WKind, SkParams, sk_begin / sk_owner, store_out4
 #include "host.cuh"
@@ -61,9 +67,15 @@ struct GvCfg {
     static constexpr int FMA_THREADS = 32 * FMA_WARPS;
     static constexpr int THREADS = 32 + FMA_THREADS;
     static constexpr int RED_BYTES = FMA_WARPS * MR * GN * 4;
-    static constexpr int STAGES_FIT = (200 * 1024 - RED_BYTES) / SLOT;
+    // split-K in a cluster: an owner receives [rank][m][GN/S columns] fp32
+    static constexpr int RBUF_BYTES = MR * GN * 4;
+    // warps that hold the CTA's summed partial (one float4 per thread)
+    static constexpr int SUM_WARPS = MR * GN / 128;
+    static constexpr int STAGES_FIT = (200 * 1024 - RED_BYTES - RBUF_BYTES) / SLOT;
     static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
-    static constexpr int SMEM_BYTES = STAGES * SLOT + RED_BYTES + 512 + 1024;
+    static constexpr int SMEM_BYTES = STAGES * SLOT + RED_BYTES + RBUF_BYTES + 512 + 1024;
+    static_assert(SUM_WARPS >= 1 && SUM_WARPS <= FMA_WARPS && MR * GN % 128 == 0,
+                  "one float4 of the summed partial per thread of the first SUM_WARPS warps");
     static_assert(STAGES >= 3, "ring");
     // The producer's transaction count is built from these sizes and the
     // launcher's boxes from GN, BK and MR: each box's bytes must be the
@@ -131,21 +143,33 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint8_t* ring = smem;                                            // STAGES x SLOT
     float* red = reinterpret_cast<float*>(ring + Cfg::STAGES * Cfg::SLOT);  // [warp][m][column]
-    uint64_t* full = reinterpret_cast<uint64_t*>(red + Cfg::FMA_WARPS * ELEMS);
+    float* rbuf = red + Cfg::FMA_WARPS * ELEMS;                      // [rank][m][column - owner * CW]
+    uint64_t* full = reinterpret_cast<uint64_t*>(rbuf + ELEMS);
     uint64_t* empty = full + Cfg::STAGES;
     uint64_t* join = empty + Cfg::STAGES;                            // the FMA warps meet
     uint64_t* flag = join + 1;                                       // ticket result published
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(flag + 1);
+    uint64_t* cl_full = flag + 1;                                    // every rank's partial arrived
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(cl_full + 1);
     volatile int* last_flag = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int G = gridDim.x;
     const int c = blockIdx.x;
-    const int u0 = sk_begin(c, p.U, G);
-    const int u1 = sk_begin(c + 1, p.U, G);
     const int KB = p.KB;
+    int u0, u1, crank = 0;                   // crank: rank in the cluster
+    if (p.S) {
+        const int tg0 = c / p.S;
+        crank = c - tg0 * p.S;
+        u0 = tg0 * KB + cl_begin(crank, KB, p.S);
+        u1 = tg0 * KB + cl_begin(crank + 1, KB, p.S);
+    } else {
+        u0 = sk_begin(c, p.U, G);
+        u1 = sk_begin(c + 1, p.U, G);
+    }
     const uint64_t limit = p.timeout_ns;
+    bool cl_waited = false;                  // this thread passed the start-up cluster barrier
+    bool cl_done = false;                    // this thread arrived on the closing cluster barrier
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -154,12 +178,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
         }
         mbar_init(join, Cfg::FMA_WARPS);
         mbar_init(flag, 1);
+        mbar_init(cl_full, 1);
+        // every rank's partial of this CTA's columns: MR x GN/S fp32 each
+        if (p.S > 1) mbar_arrive_expect_tx(cl_full, Cfg::RBUF_BYTES);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
     }
     __syncthreads();
+    // Peers store into this CTA's receive buffer and arrive on its barrier
+    // only after a cluster barrier whose arrival follows the initialisation.
+    if (p.S > 1) cluster_arrive_release();
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
@@ -339,6 +369,53 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                     acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
                 }
             if (!join_all()) break;
+            if (p.S > 1 && !whole) {
+                // Split-K in a cluster: rank o owns the CW columns
+                // [o CW, (o + 1) CW) of the group.  Thread ftid sums one
+                // float4 of the CTA's partial and stores it asynchronously
+                // into its owner's receive buffer; the owner's barrier counts
+                // the bytes.  This CTA stores into no peer after that, so it
+                // arrives on the closing cluster barrier at once.
+                const int CW = GN / p.S;
+                cluster_wait_acquire();
+                cl_waited = true;
+                if (fw < Cfg::SUM_WARPS) {
+                    const int e = ftid * 4;
+                    float4 v = *reinterpret_cast<const float4*>(red + e);
+#pragma unroll
+                    for (int w = 1; w < Cfg::FMA_WARPS; ++w) {
+                        const float4 x = *reinterpret_cast<const float4*>(red + w * ELEMS + e);
+                        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                    }
+                    const int m = e / GN, col = e - (e / GN) * GN;
+                    const int o = col / CW;
+                    st_async_v4_f32(mapa_shared(smem_u32(rbuf) + static_cast<uint32_t>(
+                                                    ((crank * MR + m) * CW + col - o * CW) * 4), o),
+                                    v, mapa_shared(smem_u32(cl_full), o));
+                }
+                cluster_arrive_release();
+                cl_done = true;
+                // owner: MR rows x CW columns, every rank's partial summed in
+                // rank order (deterministic), one float4 per thread
+                const int nq = MR * (CW >> 2);
+                if (ftid < nq) {
+                    if (!bounded_wait_cluster(cl_full, 0, abort_flag, limit, p.status)) break;
+                    const int m = ftid / (CW >> 2), c4 = ftid - m * (CW >> 2);
+                    if (m < p.M) {
+                        float4 x = *reinterpret_cast<const float4*>(rbuf + m * CW + 4 * c4);
+                        for (int r = 1; r < p.S; ++r) {
+                            const float4 y = *reinterpret_cast<const float4*>(rbuf + (r * MR + m) * CW + 4 * c4);
+                            x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+                        }
+                        float o4[4] = {x.x, x.y, x.z, x.w};
+                        if (p.relu)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o4[j] = fmaxf(o4[j], 0.f);
+                        store_out4<OUT>(p.C, p.ldc, m, t * GN + crank * CW + 4 * c4, p.N, o4);
+                    }
+                }
+                continue;
+            }
             const int jseg = c - sk_owner(t * KB, p.U, G);
             float* part = p.ws + (static_cast<long long>(t) * p.J + jseg) * ELEMS;
             for (int e = ftid * 4; e < ELEMS; e += Cfg::FMA_THREADS * 4) {
@@ -397,6 +474,27 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
         }
     }
     __syncthreads();
+    // No CTA of a cluster exits before every peer has issued its stores.
+    if (p.S > 1) {
+        if (!cl_waited) cluster_wait_acquire();
+        if (!cl_done) cluster_arrive_release();
+        cluster_wait_acquire();
+    }
+}
+
+// The cluster split of cl_split for T column groups of KB k-units, lowered
+// until the device holds all T clusters of that size at once; 0 selects
+// stream-K.  `slot` is the kernel's attribute slot (set_smem_attr done).
+template <class Cfg>
+int gemv_cluster_split(long long T, long long KB, long long cap, int num_sms, int slot) {
+    const void* k = reinterpret_cast<const void*>(gemv_kernel<Cfg>);
+    int max_s = 8;
+    for (;;) {
+        const int S = cl_split(T, KB, Cfg::GN, cap, num_sms, max_s);
+        if (S <= 1) return S;
+        if (max_active_clusters(k, slot, S, Cfg::THREADS, Cfg::SMEM_BYTES) >= T) return S;
+        max_s = S / 2;
+    }
 }
 
 template <WKind W, int MR>
@@ -405,14 +503,26 @@ int run_gemv(const GemmArgs& a) {
     int dev = 0;
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
+    auto kern = gemv_kernel<Cfg>;
+    const int slot = 40 + static_cast<int>(W) * 3 + (MR == 1 ? 0 : MR == 2 ? 1 : 2);
+    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
+        return kCudaError;
+    const long long cap = persistent_grid(di->num_sms, di->num_sms, a.ctas);
     SkPlan pl;
-    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK,
-                 static_cast<int>(persistent_grid(di->num_sms, di->num_sms, a.ctas)), &pl))
-        return kUnsupported;
-    const long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
+    if (!sk_plan(a.N, a.K, Cfg::GN, Cfg::BK, static_cast<int>(cap), &pl)) return kUnsupported;
+    long long T = pl.T, KB = pl.KB, U = pl.U, G = pl.G, J = pl.J;
+    // Split-K inside clusters where T groups times the split fill the GPU
+    // (partials meet in distributed shared memory: no workspace); else
+    // stream-K over G CTAs with a per-stream workspace.
+    const int S = gemv_cluster_split<Cfg>(T, KB, cap, di->num_sms, slot);
     int* tickets = nullptr;
     float* ws = nullptr;
-    if (!stream_workspace(dev, a.stream, T, T * J * MR * Cfg::GN * 4, &tickets, &ws)) return kCudaError;
+    if (S > 0) {
+        G = T * S;
+        J = 1;
+    } else if (!stream_workspace(dev, a.stream, T, T * J * MR * Cfg::GN * 4, &tickets, &ws)) {
+        return kCudaError;
+    }
 
     const CUtensorMapDataType at = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -430,10 +540,6 @@ int run_gemv(const GemmArgs& a) {
     }
     if (!tensor_map_2d(&tX, a.A, at, 2, a.K, a.M, a.lda * 2, 64, MR, SWZ_NONE)) return kCudaError;
 
-    auto kern = gemv_kernel<Cfg>;
-    const int slot = 40 + static_cast<int>(W) * 3 + (MR == 1 ? 0 : MR == 2 ? 1 : 2);
-    if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
-        return kCudaError;
     SkParams p;
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
@@ -443,6 +549,7 @@ int run_gemv(const GemmArgs& a) {
     p.KB = static_cast<int>(KB);
     p.U = static_cast<int>(U);
     p.J = static_cast<int>(J);
+    p.S = S;
     p.inject = inject_mode();
     p.timeout_ns = wait_limit_ns();
     p.status = device_status_ptr();
@@ -451,8 +558,23 @@ int run_gemv(const GemmArgs& a) {
     p.ws = ws;
     p.tickets = tickets;
     if (!p.status) return kCudaError;
-    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, static_cast<cudaStream_t>(a.stream)>>>(
-        tW, tS, tX, p);
+    const cudaStream_t stream = static_cast<cudaStream_t>(a.stream);
+    if (S > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(G), 1, 1);
+        cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, tW, tS, tX, p) == cudaSuccess ? kOk : kCudaError;
+    }
+    kern<<<static_cast<int>(G), Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(tW, tS, tX, p);
     return cudaGetLastError() == cudaSuccess ? kOk : kCudaError;
 }
 

@@ -379,6 +379,15 @@ __device__ __forceinline__ void st_shared_cluster_f32(uint32_t cl_addr, float v)
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cl_addr), "f"(v) : "memory");
 }
 
+// Asynchronous store of four floats into distributed shared memory: the
+// destination CTA's mbarrier at cl_bar (same CTA as cl_addr) receives a
+// complete_tx of 16 bytes, with release semantics at cluster scope, once the
+// data has landed.  The sender needs no fence.
+__device__ __forceinline__ void st_async_v4_f32(uint32_t cl_addr, float4 v, uint32_t cl_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(cl_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cl_bar) : "memory");
+}
+
 __device__ __forceinline__ void fence_acq_rel_cluster() {
     asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }
