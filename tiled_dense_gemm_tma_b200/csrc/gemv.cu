@@ -375,7 +375,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 // float4 of the CTA's partial and stores it asynchronously
                 // into its owner's receive buffer; the owner's barrier counts
                 // the bytes.  This CTA stores into no peer after that, so it
-                // arrives on the closing cluster barrier at once.
+                // arrives on the closing cluster barrier at once (relaxed: that
+                // barrier only keeps every CTA alive until all peers issued
+                // their stores; an owner reads its buffer only after its
+                // barrier counted every byte).
                 const int CW = GN / p.S;
                 cluster_wait_acquire();
                 cl_waited = true;
@@ -393,7 +396,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                                                     ((crank * MR + m) * CW + col - o * CW) * 4), o),
                                     v, mapa_shared(smem_u32(cl_full), o));
                 }
-                cluster_arrive_release();
+                cluster_arrive_relaxed();
                 cl_done = true;
                 // owner: MR rows x CW columns, every rank's partial summed in
                 // rank order (deterministic), one float4 per thread
@@ -477,7 +480,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
     // No CTA of a cluster exits before every peer has issued its stores.
     if (p.S > 1) {
         if (!cl_waited) cluster_wait_acquire();
-        if (!cl_done) cluster_arrive_release();
+        if (!cl_done) cluster_arrive_relaxed();
         cluster_wait_acquire();
     }
 }

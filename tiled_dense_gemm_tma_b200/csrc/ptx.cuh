@@ -434,6 +434,12 @@ __device__ __forceinline__ void cluster_arrive_release() {
     asm volatile("barrier.cluster.arrive.release;" ::: "memory");
 }
 
+// Arrival that orders nothing: for a barrier that only keeps the CTAs of a
+// cluster alive until every peer has passed a point.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
