@@ -13,8 +13,9 @@
 //   of all groups are cut into one contiguous, equal range per SM; a maximal
 //   run of a range inside one column group is a segment.
 // * Warp 0 streams each unit by TMA into a ring of shared-memory slots: the
-//   weight tile (128-byte swizzled rows), for 4-bit weights the unit's fp16
-//   scale row, and the activations (MR rows x 64 values per slice).
+//   weight tile (unswizzled 128-byte rows: a warp reads whole rows, which
+//   touch every bank once), for 4-bit weights the unit's fp16
+//   scale row, and the activations (MR rows x BK values).
 // * Sixteen CUDA-core warps (eight for four activation rows) read the slot:
 //   warp w takes a run of consecutive rows (vector reads fetch their
 //   activations); each lane its GN/32
@@ -52,14 +53,16 @@ struct GvCfg {
     static constexpr int MR = MR_;                      // activation rows: 1, 2 or 4
     static constexpr bool Q4 = W_ == WKind::INT4;
     static constexpr int GN = Q4 ? 256 : 128;           // columns per unit
-    static constexpr int BK = 128;                      // rows per unit (one scale group)
-    static constexpr int KSL = BK / 64;                 // 64-wide activation slices
+    // rows per unit: 4-bit units hold SG scale groups of 128 rows, so that a
+    // warp's run of rows (one group) amortises the per-unit work over more rows
+    static constexpr int BK = Q4 ? 256 : 128;
+    static constexpr int SG = BK / 128;
     static constexpr int CPL = GN / 32;                 // columns per lane
     static constexpr int W_CHUNK = BK * 128;            // one 64-column box (16-bit)
     static constexpr int W_BYTES = Q4 ? BK * GN / 2 : 2 * W_CHUNK;
-    static constexpr int S_BYTES = Q4 ? GN * 2 : 0;
-    static constexpr int X_SLICE = MR * 128;            // MR rows x 64 values
-    static constexpr int X_BYTES = KSL * X_SLICE;
+    static constexpr int S_BYTES = Q4 ? SG * GN * 2 : 0;
+    static constexpr int X_ROW = BK * 2;                // one activation row of the unit
+    static constexpr int X_BYTES = MR * X_ROW;          // MR rows x BK values
     static constexpr int SLOT = (W_BYTES + S_BYTES + X_BYTES + 1023) / 1024 * 1024;
     // 16 math warps; 8 with four activation rows (their accumulators need
     // more than the 96 registers a 544-thread CTA leaves per thread)
@@ -80,15 +83,17 @@ struct GvCfg {
     // The producer's transaction count is built from these sizes and the
     // launcher's boxes from GN, BK and MR: each box's bytes must be the
     // count it is charged.  4-bit: one (GN/2 bytes x BK rows) weight box and
-    // one (GN x 1) fp16 scale box; 16-bit: two (64 x BK) weight boxes; then
-    // KSL (64 x MR) fp16 activation boxes.  A 128-byte-swizzled box is at
-    // most 128 bytes wide and starts on a 1024-byte boundary.
+    // one (GN x SG) fp16 scale box; 16-bit: two (64 x BK) weight boxes; then
+    // one (BK x MR) 16-bit activation box (at most 256 values wide).  No box
+    // is swizzled; slots start on 1024-byte boundaries.
     static_assert(Q4 ? (W_BYTES == (GN / 2) * BK && GN / 2 == 128)
                      : (W_BYTES == 2 * W_CHUNK && W_CHUNK == 64 * 2 * BK), "weight box bytes");
-    static_assert(!Q4 || S_BYTES == GN * 2, "scale box bytes");
-    static_assert(X_SLICE == 64 * MR * 2 && X_BYTES == KSL * X_SLICE && KSL * 64 == BK,
+    static_assert(!Q4 || S_BYTES == GN * SG * 2, "scale box bytes");
+    // a warp's rows of a unit lie in one scale group
+    static_assert(!Q4 || (BK % 128 == 0 && 128 % (BK / FMA_WARPS) == 0), "rows per warp");
+    static_assert(X_ROW == BK * 2 && X_BYTES == MR * X_ROW && BK <= 256 && X_ROW % 16 == 0,
                   "activation box bytes");
-    static_assert(SLOT % 1024 == 0 && W_CHUNK % 1024 == 0, "swizzled boxes on 1024-byte boundaries");
+    static_assert(SLOT % 1024 == 0 && W_CHUNK % 1024 == 0, "boxes on 1024-byte boundaries");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -199,11 +204,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
             if constexpr (Cfg::Q4) tma_prefetch_desc(&tmS);
             uint32_t armed = 0, armed_par = 0;
             bool ok = true;
-            int it = 0;
+            int it = 0, s = 0;                               // slot s of pass ph
+            uint32_t ph = 0;
             int t = u0 / KB, kb = u0 - (u0 / KB) * KB;      // unit u = t * KB + kb
-            for (int u = u0; u < u1; ++u, ++it, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0) {
-                const int s = it % Cfg::STAGES;
-                const uint32_t ph = (it / Cfg::STAGES) & 1;
+            for (int u = u0; u < u1; ++u, ++it, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0,
+                     s = s + 1 == Cfg::STAGES ? 0 : s + 1, ph ^= s == 0) {
                 if (!bounded_wait(&empty[s], ph ^ 1, abort_flag, limit, p.status)) { ok = false; break; }
                 if (p.inject == 1 && it == 0 && c == 0) continue;   // debug: never arm slot 0
                 uint8_t* slot = ring + s * Cfg::SLOT;
@@ -211,7 +216,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 if constexpr (Cfg::Q4) {
                     mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::S_BYTES + Cfg::X_BYTES);
                     tma_load_2d(slot, &tmW, &full[s], t * (GN / 2), kb * BK);
-                    tma_load_2d(slot + Cfg::W_BYTES, &tmS, &full[s], t * GN, (kb * BK) / 128);
+                    tma_load_2d(slot + Cfg::W_BYTES, &tmS, &full[s], t * GN, kb * Cfg::SG);
                 } else {
                     // the second 64-column box is skipped when it starts past N
                     // (its columns are never stored)
@@ -220,10 +225,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                     tma_load_2d(slot, &tmW, &full[s], t * GN, kb * BK);
                     if (second) tma_load_2d(slot + Cfg::W_CHUNK, &tmW, &full[s], t * GN + 64, kb * BK);
                 }
-                // the unit's activations: KSL slices of 64 values (X_BYTES in all)
-#pragma unroll
-                for (int ks = 0; ks < Cfg::KSL; ++ks)
-                    tma_load_2d(xs + ks * Cfg::X_SLICE, &tmX, &full[s], kb * BK + 64 * ks, 0);
+                // the unit's activations: MR rows of BK values (X_BYTES)
+                tma_load_2d(xs, &tmX, &full[s], kb * BK, 0);
                 armed |= 1u << s;
                 armed_par = (armed_par & ~(1u << s)) | (ph << s);
             }
@@ -257,14 +260,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
         for (int m = 0; m < MR; ++m)
 #pragma unroll
             for (int q = 0; q < CPL; ++q) acc[m][q] = 0.f;
-        int it = 0;
+        int s = 0;                                          // slot s of pass ph
+        uint32_t ph = 0;
         int t = u0 / KB, kb = u0 - (u0 / KB) * KB;          // unit u = t * KB + kb
-        for (int u = u0; u < u1; ++u, ++it, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0) {
-            const int s = it % Cfg::STAGES;
-            const uint32_t ph = (it / Cfg::STAGES) & 1;
+        for (int u = u0; u < u1; ++u, kb = kb + 1 == KB ? 0 : kb + 1, t += kb == 0,
+                 s = s + 1 == Cfg::STAGES ? 0 : s + 1, ph ^= s == 0) {
             if (!bounded_wait(&full[s], ph, abort_flag, limit, p.status)) break;
             const uint8_t* slot = ring + s * Cfg::SLOT;
-            const uint8_t* xs = slot + Cfg::W_BYTES + Cfg::S_BYTES + (r0 >> 6) * Cfg::X_SLICE + (r0 & 63) * 2;
+            const uint8_t* xs = slot + Cfg::W_BYTES + Cfg::S_BYTES + r0 * 2;
             // activations of the warp's RPW rows: one vector read per m, kept
             // packed (two values per word) and widened where used
             uint32_t avw[MR][RPW / 2];
@@ -272,7 +275,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
             for (int m = 0; m < MR; ++m)
 #pragma unroll
                 for (int h = 0; h < RPW / 8; ++h) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(xs + m * 128 + 16 * h);
+                    const uint4 v = *reinterpret_cast<const uint4*>(xs + m * Cfg::X_ROW + 16 * h);
                     avw[m][4 * h] = v.x; avw[m][4 * h + 1] = v.y; avw[m][4 * h + 2] = v.z; avw[m][4 * h + 3] = v.w;
                 }
             auto act = [&](int m, int i) -> float {
@@ -292,10 +295,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
 #pragma unroll
                 for (int i = 0; i < RPW; ++i) {
                     const int r = r0 + i;
-                    // 4 bytes = columns 8 lane .. 8 lane + 7 of row r (16-byte
-                    // unit lane / 4, stored at unit (lane / 4) ^ (r % 8))
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                        slot + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
+                    // 4 bytes = columns 8 lane .. 8 lane + 7 of row r
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(slot + r * 128 + lane * 4);
                     const uint32_t w8 = w >> 8;
                     // pair j holds columns (j, j + 4): D = 1024 for even j, 64 for odd j
                     const uint32_t hp[4] = {nib_pair(w, kKeepLo, kSetLo), nib_pair(w, kKeepHi, kSetHi),
@@ -315,8 +316,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                         }
                     }
                 }
-                // the unit's rows share one scale group: total += s * sum_k q a
-                const uint4 sv = *reinterpret_cast<const uint4*>(slot + Cfg::W_BYTES + lane * 16);
+                // the warp's rows share one scale group: total += s * sum_k q a
+                const uint4 sv = *reinterpret_cast<const uint4*>(slot + Cfg::W_BYTES + (r0 / 128) * GN * 2 +
+                                                                 lane * 16);
                 const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
                 float sc[8];
 #pragma unroll
@@ -337,11 +339,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
 #pragma unroll
                 for (int i = 0; i < RPW; ++i) {
                     const int r = r0 + i;
-                    // 8 bytes = columns 4 lane .. 4 lane + 3: box lane / 16, 16-byte
-                    // unit (lane % 16) / 2 of the box row, stored at unit ^ (r % 8)
+                    // 8 bytes = columns 4 lane .. 4 lane + 3: box lane / 16, bytes
+                    // 8 (lane % 16) .. of the box row
                     const uint2 v = *reinterpret_cast<const uint2*>(
-                        slot + (lane >> 4) * Cfg::W_CHUNK + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) +
-                        (lane & 1) * 8);
+                        slot + (lane >> 4) * Cfg::W_CHUNK + r * 128 + (lane & 15) * 8);
                     const float2 w0 = widen2<Cfg::W>(v.x), w1 = widen2<Cfg::W>(v.y);
 #pragma unroll
                     for (int m = 0; m < MR; ++m) {
@@ -532,16 +533,16 @@ int run_gemv(const GemmArgs& a) {
     CUtensorMap tW, tS, tX;
     if constexpr (Cfg::Q4) {
         if (!tensor_map_2d(&tW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
-                           Cfg::GN / 2, Cfg::BK, SWZ_128))
+                           Cfg::GN / 2, Cfg::BK, SWZ_NONE))
             return kCudaError;
         if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128, a.lds * 2,
-                           Cfg::GN, 1, SWZ_NONE))
+                           Cfg::GN, Cfg::SG, SWZ_NONE))
             return kCudaError;
     } else {
-        if (!tensor_map_2d(&tW, a.B, at, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128)) return kCudaError;
+        if (!tensor_map_2d(&tW, a.B, at, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_NONE)) return kCudaError;
         tS = tW;                                   // unused
     }
-    if (!tensor_map_2d(&tX, a.A, at, 2, a.K, a.M, a.lda * 2, 64, MR, SWZ_NONE)) return kCudaError;
+    if (!tensor_map_2d(&tX, a.A, at, 2, a.K, a.M, a.lda * 2, Cfg::BK, MR, SWZ_NONE)) return kCudaError;
 
     SkParams p;
     p.M = static_cast<int>(a.M);
