@@ -42,8 +42,8 @@
  *   where the split does not run inside thread-block clusters, fp32 shapes
  *   with fewer 128 x 128 tiles than SMs, and 16-bit GEMMs with M > 128 whose
  *   last wave of 256 x 256 tiles is split along K).  It is allocated on the
- *   first such call
- *   on a stream (at least 8 MiB), grown when a larger call needs it (the
+ *   first such call on a stream (at least 8 MiB), grown when a larger call
+ *   needs it (the
  *   regrow frees the old one, which synchronises the device), and reused.
  *   Calls on one stream share it; calls on different streams get their own
  *   (cudaStreamPerThread counts as one stream per host thread).  A stream
@@ -202,10 +202,12 @@ TG_API tg_status tg_gemm_w4a16(int64_t M, int64_t N, int64_t K,
  *           means NaN), row pitch lds in BYTES (>= N, % 16 == 0).
  *   block_size: must be 32 (k rows per scale), else TG_ERR_UNSUPPORTED.
  *   C:      M x N bf16 output, row pitch ldc (elements, % 8 == 0).
- * Any K >= 0.  W is formed exactly as a bf16 tensor-core operand (for
- * E <= 252; a larger E overflows bf16), products accumulate in fp32, and the
- * result is rounded once to bf16.  Same status and ownership rules as
- * tg_gemm_w4a16.
+ * Any K >= 0.  For M > 4, W is formed exactly as a bf16 tensor-core
+ * operand (for E <= 252; a larger E overflows bf16); for M <= 4 the CUDA-core
+ * kernel multiplies the exact E2M1 values by the activations in fp32 and
+ * applies each 32-row block's 2^(E - 127) once per block and column.  Either
+ * way products accumulate in fp32 and the result is rounded once to bf16.
+ * Same status and ownership rules as tg_gemm_w4a16.
  */
 TG_API tg_status tg_gemm_wfp4(int64_t M, int64_t N, int64_t K,
                        const void *A, int64_t lda,
@@ -294,7 +296,7 @@ enum {
 };
 enum {
     TG_PATH_AUTO = 0,       /* the default choice by M */
-    TG_PATH_CUDA_CORE = 1,  /* CUDA-core kernel: M <= 4 only; not for FP4 weights or fp32 */
+    TG_PATH_CUDA_CORE = 1,  /* CUDA-core kernel: M <= 4 only; not for fp32 */
     TG_PATH_SMALL_M = 2,    /* weight-streaming tensor-core kernel: M <= 128 only */
     TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit and 4-bit ops) */
     TG_PATH_ONE_CTA = 4     /* persistent one-CTA tensor-core kernel (not fp32 FFMA) */

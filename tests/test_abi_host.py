@@ -277,7 +277,7 @@ def test_tuning_table_rules(lib):
         assert b.tune_query("f32_ffma", 1024, 1024)["splits"] == 3
         # malformed rules: nothing changes
         bad = [{"op": "bf16", "path": "cuda_core", "m_hi": 5},       # CUDA-core kernel: M <= 4
-               {"op": "wfp4", "path": "cuda_core", "m_hi": 4},        # no CUDA-core FP4 kernel
+               {"op": "wfp4", "path": "cuda_core", "m_hi": 5},        # CUDA-core FP4 kernel: M <= 4
                {"op": "bf16", "path": "small_m", "m_hi": 129},        # small-M kernel: M <= 128
                {"op": "f32_ffma", "path": "one_cta"},                 # fp32 FFMA has one kernel
                {"op": "bf16", "splits": 2},                           # split count: FFMA only

@@ -56,6 +56,17 @@ def _run4(tg, A, Bq, S, N, relu=False):
     return from_dev(C, "f16")
 
 
+def _runfp4(tg, A, Bq, E, N, relu=False):
+    import torch
+    M = A.shape[0]
+    big, C, pad = guarded_out(M, N, "bf16")
+    tg.gemm_wfp4(to_dev(A, "bf16"), to_dev(Bq, "u8"), to_dev(E, "u8"), N, C=C, relu=relu)
+    torch.cuda.synchronize()
+    assert tg.last_device_status() == 0
+    check_guard(big, "bf16", M, N, pad)
+    return from_dev(C, "bf16")
+
+
 SHAPES16 = [(1, 1, 1), (1, 8, 127), (2, 255, 129), (3, 257, 2048), (4, 1000, 5000),
             (1, 4104, 300), (4, 8192, 1024), (2, 520, 8192)]
 
@@ -119,7 +130,7 @@ def test_gemv_w4a16_bit_exact_groups_and_repeatable(tg):
 CLUSTER_SHAPES = [(1, 8000, 1280), (3, 8192, 640), (4, 4000, 1024), (2, 8192, 8192)]
 
 
-@pytest.mark.parametrize("kind", ["w4a16", "bf16", "f16"])
+@pytest.mark.parametrize("kind", ["w4a16", "wfp4", "bf16", "f16"])
 @pytest.mark.parametrize("shape", CLUSTER_SHAPES)
 def test_gemv_cluster_and_stream_k_splits(tg, kind, shape):
     # These shapes give T column groups x a split S of 2 to 8 that fill the
@@ -134,6 +145,11 @@ def test_gemv_cluster_and_stream_k_splits(tg, kind, shape):
         ref = oracle.gemm_w4a16(A, Bq, S, N=N, relu=True)
         run = lambda: _run4(tg, A, Bq, S, N, relu=True)
         frob = 2e-3
+    elif kind == "wfp4":
+        A, Bq, E, _ = synth.wfp4(M, N, K, seed=5)
+        ref = oracle.gemm_wfp4(A, Bq, E, N=N, relu=True)
+        run = lambda: _runfp4(tg, A, Bq, E, N, relu=True)
+        frob = FROB["bf16"]
     else:
         K = K - 24                                   # ragged in K
         A, B = synth.normal(M, N, K, seed=5, dtype=kind, scale_by_sqrt_k=True)
@@ -149,6 +165,61 @@ def test_gemv_cluster_and_stream_k_splits(tg, kind, shape):
         finally:
             tg.tune_set([])
         assert np.array_equal(first, again)
-        got = decode16(first, "f16" if kind == "w4a16" else kind)
+        got = decode16(first, {"w4a16": "f16", "wfp4": "bf16"}.get(kind, kind))
         assert_close(got, ref, RTOL, ATOL, f"{kind} {shape} ctas={ctas}")
         assert rel_frob(got, ref) <= frob
+
+
+SHAPESFP4 = [(1, 256, 256), (2, 301, 96), (3, 520, 200), (4, 1000, 544), (1, 4104, 300),
+             (2, 8192, 1024)]
+
+
+@pytest.mark.parametrize("shape", SHAPESFP4)
+@pytest.mark.parametrize("relu", [False, True])
+def test_gemv_wfp4(tg, shape, relu):
+    # FP4 weights (E2M1 codes, one E8M0 scale per 32 rows and column) on the
+    # CUDA-core kernel: ragged N (odd, not a multiple of 256), K not a
+    # multiple of the 32-row block or of the 256-row unit
+    M, N, K = shape
+    A, Bq, E, _ = synth.wfp4(M, N, K, seed=6)
+    got = decode16(_runfp4(tg, A, Bq, E, N, relu), "bf16")
+    ref = oracle.gemm_wfp4(A, Bq, E, N=N, relu=relu)
+    assert_close(got, ref, RTOL, ATOL, f"wfp4 {shape} relu={relu}")
+    assert rel_frob(got, ref) <= FROB["bf16"]
+
+
+@pytest.mark.parametrize("M", [1, 3, 4])
+def test_gemv_wfp4_bit_exact_scales_and_repeatable(tg, M):
+    # integer activations in {-2..2} and every code: with scales 2^-3 .. 2^2
+    # every partial sum is a multiple of 2^-4 below 2^14, and with the
+    # smallest scales (E = 0, the subnormal 2^-127; E = 1, 2) a multiple of
+    # 2^-128 below 2^-113: exact in fp32 either way, so C is the exact result
+    # rounded once to bf16 (a subnormal bf16 in the second case)
+    N, K = 1000, 320
+    A, Bq, _, _ = synth.wfp4(M, N, K, seed=7, a_int=2)
+    rng = np.random.default_rng(7)
+    for lo, hi in ((124, 130), (0, 3)):
+        E = rng.integers(lo, hi, size=((K + 31) // 32, N)).astype(np.uint8)
+        got = _runfp4(tg, A, Bq, E, N)
+        ref = oracle.gemm_wfp4(A, Bq, E, N=N)
+        assert np.array_equal(decode16(got, "bf16"), decode16(oracle.round_bf16(ref), "bf16")), (lo, hi)
+    A, Bq, E, _ = synth.wfp4(M, 8192, 8192, seed=4)
+    first = _runfp4(tg, A, Bq, E, 8192)
+    for _ in range(3):
+        assert np.array_equal(_runfp4(tg, A, Bq, E, 8192), first)
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_gemv_wfp4_nan_scale(tg, M):
+    # an E8M0 byte of 255 is NaN: exactly the columns with such a block are NaN
+    N, K = 264, 128
+    A, Bq, E, _ = synth.wfp4(M, N, K, seed=8)
+    E = E.copy()
+    E[1, 5] = 255
+    E[3, 200] = 255
+    got = decode16(_runfp4(tg, A, Bq, E, N), "bf16")
+    ref = oracle.gemm_wfp4(A, Bq, E, N=N)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert set(np.where(np.isnan(got).any(axis=0))[0]) == {5, 200}
+    ok = ~np.isnan(ref)
+    assert_close(got[ok], ref[ok], RTOL, ATOL, "non-NaN columns")

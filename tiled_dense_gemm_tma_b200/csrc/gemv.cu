@@ -51,16 +51,22 @@ template <WKind W_, int MR_>
 struct GvCfg {
     static constexpr WKind W = W_;
     static constexpr int MR = MR_;                      // activation rows: 1, 2 or 4
-    static constexpr bool Q4 = W_ == WKind::INT4;
+    static constexpr bool I4 = W_ == WKind::INT4;      // signed 4-bit integers, fp16 group scales
+    static constexpr bool F4 = W_ == WKind::FP4;       // E2M1 codes, E8M0 block scales
+    static constexpr bool Q4 = I4 || F4;               // packed two per byte
+    static constexpr WKind ACT = I4 ? WKind::F16 : F4 ? WKind::BF16 : W_;   // activations and C
     static constexpr int GN = Q4 ? 256 : 128;           // columns per unit
-    // rows per unit: 4-bit units hold SG scale groups of 128 rows, so that a
-    // warp's run of rows (one group) amortises the per-unit work over more rows
+    // rows per unit: 4-bit units hold SG scale groups of 128 rows (integer
+    // weights) or SB blocks of 32 rows (FP4), so that a warp's run of rows (in
+    // one group or block) amortises the per-unit work over more rows
     static constexpr int BK = Q4 ? 256 : 128;
     static constexpr int SG = BK / 128;
+    static constexpr int SB = BK / 32;
+    static constexpr int S_ROWS = I4 ? SG : SB;        // scale rows of a unit
     static constexpr int CPL = GN / 32;                 // columns per lane
     static constexpr int W_CHUNK = BK * 128;            // one 64-column box (16-bit)
     static constexpr int W_BYTES = Q4 ? BK * GN / 2 : 2 * W_CHUNK;
-    static constexpr int S_BYTES = Q4 ? SG * GN * 2 : 0;
+    static constexpr int S_BYTES = I4 ? SG * GN * 2 : F4 ? SB * GN : 0;
     static constexpr int X_ROW = BK * 2;                // one activation row of the unit
     static constexpr int X_BYTES = MR * X_ROW;          // MR rows x BK values
     static constexpr int SLOT = (W_BYTES + S_BYTES + X_BYTES + 1023) / 1024 * 1024;
@@ -83,14 +89,15 @@ struct GvCfg {
     // The producer's transaction count is built from these sizes and the
     // launcher's boxes from GN, BK and MR: each box's bytes must be the
     // count it is charged.  4-bit: one (GN/2 bytes x BK rows) weight box and
-    // one (GN x SG) fp16 scale box; 16-bit: two (64 x BK) weight boxes; then
+    // one (GN x SG) fp16 scale box (FP4: (GN x SB) E8M0 bytes); 16-bit: two
+    // (64 x BK) weight boxes; then
     // one (BK x MR) 16-bit activation box (at most 256 values wide).  No box
     // is swizzled; slots start on 1024-byte boundaries.
     static_assert(Q4 ? (W_BYTES == (GN / 2) * BK && GN / 2 == 128)
                      : (W_BYTES == 2 * W_CHUNK && W_CHUNK == 64 * 2 * BK), "weight box bytes");
-    static_assert(!Q4 || S_BYTES == GN * SG * 2, "scale box bytes");
-    // a warp's rows of a unit lie in one scale group
-    static_assert(!Q4 || (BK % 128 == 0 && 128 % (BK / FMA_WARPS) == 0), "rows per warp");
+    static_assert(!Q4 || S_BYTES == GN * S_ROWS * (I4 ? 2 : 1), "scale box bytes");
+    // a warp's rows of a unit lie in one scale group (block)
+    static_assert(!Q4 || (BK % 128 == 0 && (I4 ? 128 : 32) % (BK / FMA_WARPS) == 0), "rows per warp");
     static_assert(X_ROW == BK * 2 && X_BYTES == MR * X_ROW && BK <= 256 && X_ROW % 16 == 0,
                   "activation box bytes");
     static_assert(SLOT % 1024 == 0 && W_CHUNK % 1024 == 0, "boxes on 1024-byte boundaries");
@@ -127,6 +134,50 @@ __device__ __forceinline__ void add_f16_f32(float& d, unsigned short x) {
     asm("add.rn.f32.f16 %0, %1, %0;" : "+f"(d) : "h"(x));
 }
 
+// Paired fp32 arithmetic (two independent IEEE operations per instruction,
+// each rounded as its scalar form).
+__device__ __forceinline__ uint64_t pk(float x, float y) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ void fma2(uint64_t& d, uint64_t x, uint64_t y) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(x), "l"(y));
+}
+
+// The two E2M1 codes of the low byte of x (low nibble first) as an fp32
+// pair: the hardware conversion to an fp16 pair is exact (every E2M1 value
+// has at most two significant bits), and so is the widening.
+__device__ __forceinline__ uint64_t e2m1_pair_f32(uint32_t x) {
+    uint64_t r;
+    asm("{\n\t.reg .b8 c;\n\t.reg .b32 h;\n\t.reg .f16 lo, hi;\n\t.reg .f32 flo, fhi;\n\t"
+        "cvt.u8.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h, c;\n\t"
+        "mov.b32 {lo, hi}, h;\n\t"
+        "cvt.f32.f16 flo, lo;\n\t"
+        "cvt.f32.f16 fhi, hi;\n\t"
+        "mov.b64 %0, {flo, fhi};\n\t}"
+        : "=l"(r) : "r"(x));
+    return r;
+}
+
+// fp32 factors 2^(E - 127) of the four E8M0 bytes of e: the byte shifted
+// into the exponent field; E = 0 is the subnormal 2^-127 and E = 255 NaN,
+// both formed by the fraction bit 0x00400000.
+__device__ __forceinline__ void e8m0_factors(uint32_t e, float* f) {
+    const uint32_t special = __vcmpeq4(e, 0u) | __vcmpeq4(e, 0xFFFFFFFFu);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const uint32_t eb = (e >> (8 * b)) & 0xFFu;
+        f[b] = __uint_as_float((eb << 23) | ((special >> (8 * b)) & 1u ? 0x00400000u : 0u));
+    }
+}
+
 // Two activations (or 16-bit weights) packed in a word, widened to fp32.
 template <WKind T>
 __device__ __forceinline__ float2 widen2(uint32_t w) {
@@ -141,7 +192,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
             const __grid_constant__ CUtensorMap tmX,
             const SkParams p) {
     constexpr int MR = Cfg::MR, GN = Cfg::GN, CPL = Cfg::CPL, BK = Cfg::BK;
-    constexpr WKind OUT = Cfg::Q4 ? WKind::F16 : Cfg::W;    // output / activation type
+    constexpr WKind OUT = Cfg::ACT;                          // output / activation type
     constexpr int ELEMS = MR * GN;                           // one segment's sums
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -216,7 +267,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 if constexpr (Cfg::Q4) {
                     mbar_arrive_expect_tx(&full[s], Cfg::W_BYTES + Cfg::S_BYTES + Cfg::X_BYTES);
                     tma_load_2d(slot, &tmW, &full[s], t * (GN / 2), kb * BK);
-                    tma_load_2d(slot + Cfg::W_BYTES, &tmS, &full[s], t * GN, kb * Cfg::SG);
+                    tma_load_2d(slot + Cfg::W_BYTES, &tmS, &full[s], t * GN, kb * Cfg::S_ROWS);
                 } else {
                     // the second 64-column box is skipped when it starts past N
                     // (its columns are never stored)
@@ -282,7 +333,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                 const float2 f = widen2<OUT>(avw[m][i >> 1]);
                 return (i & 1) ? f.y : f.x;
             };
-            if constexpr (Cfg::Q4) {
+            if constexpr (Cfg::I4) {
                 // f sums per column (nibble j of the lane's word is column j)
                 float fac[MR][CPL];
                 float suma[MR];
@@ -333,6 +384,43 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmW,
                     for (int j = 0; j < CPL; ++j) {
                         const float d = (j & 1) ? 64.f : 1024.f;
                         acc[m][j] = fmaf(sc[j], fmaf(d, fac[m][j], -(d + 8.f) * suma[m]), acc[m][j]);
+                    }
+                }
+            } else if constexpr (Cfg::F4) {
+                // column pairs (2j, 2j + 1) = byte j of the lane's word
+                uint64_t fac[MR][CPL / 2];
+#pragma unroll
+                for (int m = 0; m < MR; ++m)
+#pragma unroll
+                    for (int q = 0; q < CPL / 2; ++q) fac[m][q] = 0ull;
+#pragma unroll
+                for (int i = 0; i < RPW; ++i) {
+                    const int r = r0 + i;
+                    // 4 bytes = columns 8 lane .. 8 lane + 7 of row r
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(slot + r * 128 + lane * 4);
+                    uint64_t f2[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) f2[j] = e2m1_pair_f32(w >> (8 * j));
+#pragma unroll
+                    for (int m = 0; m < MR; ++m) {
+                        const float am = act(m, i);
+                        const uint64_t a2 = pk(am, am);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) fma2(fac[m][j], f2[j], a2);
+                    }
+                }
+                // the warp's rows share one 32-row block: total += 2^(E - 127) * sum_k v a
+                const uint2 ev = *reinterpret_cast<const uint2*>(slot + Cfg::W_BYTES + (r0 / 32) * GN + lane * 8);
+                float sc[8];
+                e8m0_factors(ev.x, sc);
+                e8m0_factors(ev.y, sc + 4);
+#pragma unroll
+                for (int m = 0; m < MR; ++m) {
+#pragma unroll
+                    for (int j = 0; j < CPL / 2; ++j) {
+                        const float2 f = upk(fac[m][j]);
+                        acc[m][2 * j] = fmaf(sc[2 * j], f.x, acc[m][2 * j]);
+                        acc[m][2 * j + 1] = fmaf(sc[2 * j + 1], f.y, acc[m][2 * j + 1]);
                     }
                 }
             } else {
@@ -508,7 +596,7 @@ int run_gemv(const GemmArgs& a) {
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
     auto kern = gemv_kernel<Cfg>;
-    const int slot = 40 + static_cast<int>(W) * 3 + (MR == 1 ? 0 : MR == 2 ? 1 : 2);
+    const int slot = (W == WKind::FP4 ? 58 : 40 + static_cast<int>(W) * 3) + (MR == 1 ? 0 : MR == 2 ? 1 : 2);
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
         return kCudaError;
     const long long cap = persistent_grid(di->num_sms, di->num_sms, a.ctas);
@@ -528,16 +616,18 @@ int run_gemv(const GemmArgs& a) {
         return kCudaError;
     }
 
-    const CUtensorMapDataType at = W == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUtensorMapDataType at = Cfg::ACT == WKind::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tW, tS, tX;
     if constexpr (Cfg::Q4) {
         if (!tensor_map_2d(&tW, a.B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (a.N + 1) / 2, a.K, a.ldb,
                            Cfg::GN / 2, Cfg::BK, SWZ_NONE))
             return kCudaError;
-        if (!tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128, a.lds * 2,
-                           Cfg::GN, Cfg::SG, SWZ_NONE))
-            return kCudaError;
+        const bool ok = Cfg::I4 ? tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.K / 128,
+                                                a.lds * 2, Cfg::GN, Cfg::SG, SWZ_NONE)
+                                : tensor_map_2d(&tS, a.scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, (a.K + 31) / 32,
+                                                a.lds, Cfg::GN, Cfg::SB, SWZ_NONE);
+        if (!ok) return kCudaError;
     } else {
         if (!tensor_map_2d(&tW, a.B, at, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_NONE)) return kCudaError;
         tS = tW;                                   // unused
@@ -594,5 +684,6 @@ int dispatch_gemv(const GemmArgs& a) {
 int launch_gemv_bf16(const GemmArgs& a) { return dispatch_gemv<WKind::BF16>(a); }
 int launch_gemv_f16(const GemmArgs& a) { return dispatch_gemv<WKind::F16>(a); }
 int launch_gemv_w4a16(const GemmArgs& a) { return dispatch_gemv<WKind::INT4>(a); }
+int launch_gemv_wfp4(const GemmArgs& a) { return dispatch_gemv<WKind::FP4>(a); }
 
 }  // namespace tg

@@ -69,6 +69,7 @@ int launch_skinny_trans_b(const GemmArgs& a, int bf16);
 int launch_gemv_bf16(const GemmArgs& a);
 int launch_gemv_f16(const GemmArgs& a);
 int launch_gemv_w4a16(const GemmArgs& a);
+int launch_gemv_wfp4(const GemmArgs& a);
 void mark_workspaces_dirty(int dev);
 // The argument checks every 16-bit and fp32 entry point runs before any CUDA
 // call (sizes, pointers, leading dimensions, the row-pitch bound, alignment)

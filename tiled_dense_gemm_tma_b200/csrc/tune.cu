@@ -47,7 +47,7 @@ bool tune_rule_valid(const TuneRule& r) {
         return false;
     switch (r.path) {
         case PATH_AUTO: return true;
-        case PATH_CUDA_CORE: return !fp32 && r.op != OP_WFP4 && r.m_hi <= 4;
+        case PATH_CUDA_CORE: return !fp32 && r.m_hi <= 4;
         case PATH_SMALL_M: return !fp32 && r.m_hi <= 128;
         case PATH_CTA_PAIR: return !fp32;
         case PATH_ONE_CTA: return r.op != OP_F32_FFMA;
