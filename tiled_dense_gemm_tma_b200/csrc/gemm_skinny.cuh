@@ -27,9 +27,11 @@
 //   in {8, 4, 2, 1} fill at least three quarters of the SMs): group t goes to
 //   the S CTAs of cluster t, each taking a contiguous part of its k-units.
 //   When its accumulator is final a CTA's ring is idle; the ranks exchange
-//   "ring free" signals, write their partials of each rank's GN/S columns
-//   into that rank's ring through distributed shared memory, and each rank
-//   sums its columns' S partials in rank order (deterministic) and writes C.
+//   "ring free" signals, store their partials of each rank's GN/S columns
+//   into that rank's ring through distributed shared memory (st.async: the
+//   owner's mbarrier counts the bytes, so no sender waits on a fence), and
+//   each rank sums its columns' S partials in rank order (deterministic) and
+//   writes C.
 //   No global round trips (partials, fences, tickets) sit between the last
 //   MMA and the output, which is where stream-K spends its tail.
 // * Weights arrive either as fp16/bf16 tiles by TMA, or as packed 4-bit
@@ -234,6 +236,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
     }
     const uint64_t limit = p.timeout_ns;
     bool cl_waited = false;                  // this thread passed the start-up cluster barrier
+    bool cl_done = false;                    // this thread arrived on the closing cluster barrier
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
@@ -253,7 +256,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
         mbar_init(epi_bar, Cfg::EPI_WARPS);
         mbar_init(flag_bar, 1);
         mbar_init(cl_ready, p.S > 1 ? p.S - 1 : 1);
-        mbar_init(cl_full, Cfg::EPI_WARPS * Cfg::NSUB);
+        mbar_init(cl_full, 1);
+        // every rank's partial of this CTA's GN/S columns, rows m < M, fp32
+        if (p.S > 1) mbar_arrive_expect_tx(cl_full, static_cast<uint32_t>(p.M) * Cfg::GN * 4);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -444,7 +449,7 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 cl_waited = true;
                 if (etid == 0) {
                     // the copy engine's and the tensor core's accesses to the
-                    // ring are complete; the peers' plain stores come next
+                    // ring are complete; the peers' stores come next
                     fence_proxy_async_smem();
                     for (int pr = 0; pr < p.S; ++pr)
                         if (pr != crank) mbar_arrive_relaxed_cluster(mapa_shared(smem_u32(cl_ready), pr));
@@ -494,9 +499,10 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                         const int o = nj / CW;
                         const uint32_t dst = mapa_shared(
                             smem_u32(ring) + static_cast<uint32_t>(((crank * Cfg::MPAD + mc) * CW + nj - o * CW) * 4), o);
+                        const uint32_t obar = mapa_shared(smem_u32(cl_full), o);
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            if (mc + i < p.M) st_shared_cluster_f32(dst + i * CW * 4, __uint_as_float(v[i]));
+                            if (mc + i < p.M) st_async_b32(dst + i * CW * 4, v[i], obar);
                     } else {
                         float* col = slot + nj;
 #pragma unroll
@@ -506,15 +512,12 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
                 }
             }
             if (cl) {
-                // the warp's 32 columns of sub-tile j belong to one owner:
-                // one fence for all the warp's stores, one arrive per sub-tile
-                fence_acq_rel_cluster();
-                __syncwarp();
-                if (lane == 0)
-#pragma unroll
-                    for (int j = 0; j < Cfg::NSUB; ++j)
-                        mbar_arrive_release_cluster(
-                            mapa_shared(smem_u32(cl_full), (j * Cfg::TN + q * 32) / CW));
+                // This thread stores into no peer after this: arrive on the
+                // closing cluster barrier now (relaxed: it only keeps every
+                // CTA alive until all peers issued their stores; the owners
+                // read their rings after their barriers counted every byte).
+                cluster_arrive_relaxed();
+                cl_done = true;
             }
             tc_fence_before();
             __syncwarp();
@@ -661,9 +664,9 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (p.S > 1) {
-        // no CTA leaves while a peer may still write into its shared memory
+        // no CTA leaves before every peer has issued its stores
         if (!cl_waited) cluster_wait_acquire();
-        cluster_arrive_release();
+        if (!cl_done) cluster_arrive_relaxed();
         cluster_wait_acquire();
     }
 }

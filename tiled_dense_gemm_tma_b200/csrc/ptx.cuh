@@ -371,12 +371,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
 // ------------------------------------------- split-K reduction in a cluster
 //
 // Partial sums travel between the CTAs of a cluster through distributed
-// shared memory: plain stores to a peer's shared memory, then an arrive on an
-// mbarrier of that peer with release semantics at cluster scope; the peer
-// waits with acquire semantics at cluster scope and then reads the data.
+// shared memory: asynchronous stores into a peer's shared memory, each
+// completing its bytes on an mbarrier of that peer (release semantics at
+// cluster scope); the peer, having announced the byte count, waits with
+// acquire semantics at cluster scope and then reads the data.
 
-__device__ __forceinline__ void st_shared_cluster_f32(uint32_t cl_addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cl_addr), "f"(v) : "memory");
+// Asynchronous store of one 32-bit word into distributed shared memory,
+// completing 4 bytes on the destination CTA's mbarrier at cl_bar (as
+// st_async_v4_f32 below).
+__device__ __forceinline__ void st_async_b32(uint32_t cl_addr, uint32_t v, uint32_t cl_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(cl_addr), "r"(v), "r"(cl_bar) : "memory");
 }
 
 // Asynchronous store of four floats into distributed shared memory: the
@@ -388,17 +393,9 @@ __device__ __forceinline__ void st_async_v4_f32(uint32_t cl_addr, float4 v, uint
                  ::"r"(cl_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cl_bar) : "memory");
 }
 
-__device__ __forceinline__ void fence_acq_rel_cluster() {
-    asm volatile("fence.acq_rel.cluster;" ::: "memory");
-}
-
 // Arrive with no ordering of this thread's earlier accesses (a pure signal).
 __device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cl_addr) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cl_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
