@@ -8,9 +8,11 @@ ring slot: a barrier that nothing then completes.  TG_DEBUG_TIMEOUT_US=200000
 bounds every barrier wait at 0.2 s.  That CTA gives up, records the timeout
 in the device status word, drains its in-flight copies, frees its tensor
 memory and exits; the other CTAs finish their work.  In the kernels that
-split K across CTAs (weight-streaming small-M, CUDA-core M <= 4, fp32 FFMA
-split-K) the tiles CTA 0 contributes to are then left with incomplete
-tickets, so the status read must mark the split-K workspace for re-zeroing:
+split K across CTAs through global memory (weight-streaming small-M and
+CUDA-core M <= 4 under stream-K, fp32 FFMA split-K) the tiles CTA 0
+contributes to are then left with incomplete tickets, so the status read
+must mark the split-K workspace for re-zeroing (inside a cluster, CTA 0's
+peers time out on the partials it never sends and exit with it):
 the second call of the same shape on the same stream must match the fp64
 oracle.  Each family runs in a child process because both knobs are read once
 per process; the one-CTA fallback kernels run with TG_NO_PAIR=1 as well.
@@ -58,9 +60,10 @@ CHILD = textwrap.dedent("""
             call = lambda: tg.gemm_f32(dA, dB, mode=mode)
             conv = lambda C: from_dev(C, "f32")
             tol = None
-        elif fam.startswith("w4a16") or fam.startswith("skinny_w4a16") or fam == "gemv_w4a16":
+        elif fam.startswith("w4a16") or fam.startswith("skinny_w4a16") or fam.startswith("gemv_w4a16"):
             M, N, K = {"w4a16_pair": (512, 1024, 1024), "w4a16_large": (512, 1024, 1024),
-                       "skinny_w4a16": (16, 2048, 4096), "gemv_w4a16": (2, 2048, 8192)}[fam]
+                       "skinny_w4a16": (16, 2048, 4096), "gemv_w4a16": (2, 2048, 8192),
+                       "gemv_w4a16_cluster": (1, 8192, 8192)}[fam]
             A, Bq, S, _ = synth.w4a16(M, N, K, seed=4)
             dA, dB, dS = to_dev(A, "f16"), to_dev(Bq, "u8"), to_dev(S, "f16")
             ref = oracle.gemm_w4a16(A, Bq, S, N=N)
@@ -76,7 +79,8 @@ CHILD = textwrap.dedent("""
             tol = (1e-2, 1e-2)
         else:
             M, N, K = {"wfp4_pair": (512, 1024, 1024), "wfp4_large": (512, 1024, 1024),
-                       "skinny_wfp4": (16, 2048, 4096)}[fam]
+                       "skinny_wfp4": (16, 2048, 4096), "gemv_wfp4": (3, 2048, 4096),
+                       "gemv_wfp4_cluster": (2, 8192, 1024)}[fam]
             A, Bq, E, _ = synth.wfp4(M, N, K, seed=4)
             dA, dB, dE = to_dev(A, "bf16"), to_dev(Bq, "u8"), to_dev(E, "u8")
             ref = oracle.gemm_wfp4(A, Bq, E, N=N)
@@ -105,9 +109,12 @@ CHILD = textwrap.dedent("""
     print("RESULT", st, st2, st3, x, round(dt, 3))
 """) % (ROOT, os.path.join(ROOT, "tests"))
 
+# gemv_*_cluster: shapes whose CUDA-core split runs inside clusters (the
+# owners' byte-counting barriers and the closing cluster barrier abort too)
 FAMILIES = ["tc2_bf16", "tf32", "skinny_bf16", "skinny_bf16_tb", "gemv_bf16", "ffma",
-            "ffma_splitk", "w4a16_pair", "skinny_w4a16", "gemv_w4a16", "wfp4_pair",
-            "skinny_wfp4", "sp24_pair", "tc_bf16", "w4a16_large", "wfp4_large", "sp24_one"]
+            "ffma_splitk", "w4a16_pair", "skinny_w4a16", "gemv_w4a16", "gemv_w4a16_cluster",
+            "wfp4_pair", "skinny_wfp4", "gemv_wfp4", "gemv_wfp4_cluster", "sp24_pair", "tc_bf16",
+            "w4a16_large", "wfp4_large", "sp24_one"]
 # run with the CTA-pair kernels off
 ONE_CTA = {"tc_bf16", "w4a16_large", "wfp4_large", "sp24_one"}
 
