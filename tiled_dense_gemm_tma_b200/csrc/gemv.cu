@@ -14,18 +14,21 @@
 //   run of a range inside one column group is a segment.
 // * Warp 0 streams each unit by TMA into a ring of shared-memory slots: the
 //   weight tile (unswizzled 128-byte rows: a warp reads whole rows, which
-//   touch every bank once), for 4-bit weights the unit's fp16
-//   scale row, and the activations (MR rows x BK values).
+//   touch every bank once), for 4-bit weights the unit's scale rows (fp16
+//   group scales, or E8M0 block exponents for FP4), and the activations
+//   (MR rows x BK values).
 // * Sixteen CUDA-core warps (eight for four activation rows) read the slot:
 //   warp w takes a run of consecutive rows (vector reads fetch their
-//   activations); each lane its GN/32
-//   neighbouring columns of a row.  16-bit weights widen exactly to fp32 and
-//   multiply into fp32 accumulators.  Signed 4-bit weights decode exactly,
-//   two per logic op, into fp16 pairs (nib_pair); mixed-precision FMAs (fp16
-//   inputs, fp32 accumulator) form per unit and lane sum_k q[k][n] a[k] in
-//   fp32, which the group scale s[g][n] multiplies once per unit (the
+//   activations), each lane its GN/32 neighbouring columns of a row.
+//   16-bit weights widen exactly to fp32 and multiply into fp32
+//   accumulators.  Signed 4-bit weights decode exactly, two per logic op,
+//   into fp16 pairs (nib_pair); mixed-precision FMAs (fp16 inputs, fp32
+//   accumulator) form per warp and lane sum_k q[k][n] a[k] over the warp's
+//   rows in fp32, which the group scale s[g][n] multiplies once (the
 //   dequantised weight W = q * s of the pages' dequantize GEMM, with the
-//   scale factored out of the unit's sum).
+//   scale factored out of the sum).  FP4 codes become exact fp16 pairs by
+//   the hardware conversion, are widened to fp32 and multiplied with paired
+//   fp32 FMAs; the block's 2^(E - 127) is applied once per warp and column.
 // * At a segment's end the warps' sums are added in warp order through
 //   shared memory.  A segment that covers its whole column group writes C.
 //   In a cluster, rank o owns GN/S columns of the group: every rank stores
@@ -90,9 +93,9 @@ struct GvCfg {
     // launcher's boxes from GN, BK and MR: each box's bytes must be the
     // count it is charged.  4-bit: one (GN/2 bytes x BK rows) weight box and
     // one (GN x SG) fp16 scale box (FP4: (GN x SB) E8M0 bytes); 16-bit: two
-    // (64 x BK) weight boxes; then
-    // one (BK x MR) 16-bit activation box (at most 256 values wide).  No box
-    // is swizzled; slots start on 1024-byte boundaries.
+    // (64 x BK) weight boxes; then one (BK x MR) 16-bit activation box (at
+    // most 256 values wide).  No box is swizzled; slots start on 1024-byte
+    // boundaries.
     static_assert(Q4 ? (W_BYTES == (GN / 2) * BK && GN / 2 == 128)
                      : (W_BYTES == 2 * W_CHUNK && W_CHUNK == 64 * 2 * BK), "weight box bytes");
     static_assert(!Q4 || S_BYTES == GN * S_ROWS * (I4 ? 2 : 1), "scale box bytes");
@@ -112,8 +115,8 @@ struct GvCfg {
 // significant bits, so f * a is exact in fp32 for an fp16 activation a, and
 //     sum_k q[k] a[k] = D sum_k f[k] a[k] - (D + 8) sum_k a[k].
 // One lop3 keeps the nibbles at bits p and p + 16 of x, flips their bit 3
-// and sets the exponent of 1.0 in both halves: per bit, lanes of `keep`
-// take x (xor the flip bit of `set`), the rest take `set`.
+// and sets the exponent of 1.0 in both halves: a bit set in `keep` takes x's
+// bit (inverted where `set` has it set), any other bit takes `set`'s.
 __device__ __forceinline__ uint32_t nib_pair(uint32_t x, uint32_t keep, uint32_t set) {
     uint32_t r;
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(x), "r"(keep), "r"(set));
