@@ -23,6 +23,13 @@ template <int FMT, OutT OUT>
 using Cfg2T01 = Tc2Cfg<FMT, OUT, 6, 0, 0>;
 template <int FMT, OutT OUT>
 using Cfg2T11 = Tc2Cfg<FMT, OUT, 6, 1, 0>;
+// Operand-swapped CTA pair for M <= 128 (C^T = B^T A^T, 128-column pair tiles,
+// written transposed): B^T arrives from B stored K x N (MN-major) or N x K
+// (K-major); A^T is A stored M x K, read K-major.
+template <int FMT, OutT OUT>
+using Cfg2S = Tc2Cfg<FMT, OUT, 6, 1, 0, 128, 1>;
+template <int FMT, OutT OUT>
+using Cfg2ST = Tc2Cfg<FMT, OUT, 6, 0, 0, 128, 1>;
 
 template <class Cfg>
 int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, int slot) {
@@ -88,7 +95,11 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     if (Cfg::B_MN ? !tensor_map_2d(&tB, a.B, dt, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128)
                   : !tensor_map_2d(&tB, a.B, dt, 2, a.K, a.N, a.ldb * 2, Cfg::BK, Cfg::HN, SWZ_128))
         return kCudaError;
-    if (!tensor_map_2d(&tC, a.C, dt, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
+    // C: 64-column x 32-row boxes of the tile; in the operand-swapped mode the
+    // kernel's M x N is C^T, and C (a.N rows x a.M columns) takes unswizzled
+    // boxes of 32 columns x 64 rows
+    if (Cfg::TOUT ? !tensor_map_2d(&tC, a.C, dt, 2, a.M, a.N, a.ldc * 2, 32, 64, SWZ_NONE)
+                  : !tensor_map_2d(&tC, a.C, dt, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
         return kCudaError;
     auto kern = tc2_gemm_kernel<Cfg>;
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
@@ -152,9 +163,25 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
 
 }  // namespace
 
+// The CTA-pair kernel for M <= 128 with the operands swapped: the kernel's
+// A is B^T (its M = N) and its B is A^T (its N = M); C is written transposed
+// back.  trans_b: B is stored N x K.
+template <int FMT, OutT OUT>
+int run_pair_swapped(const GemmArgs& a, CUtensorMapDataType dt, int trans_b, int slot) {
+    GemmArgs s = a;
+    s.M = a.N;
+    s.N = a.M;
+    s.A = a.B;
+    s.lda = a.ldb;
+    s.B = a.A;
+    s.ldb = a.lda;
+    return trans_b ? run_pair<Cfg2ST<FMT, OUT>>(s, dt, slot + 1) : run_pair<Cfg2S<FMT, OUT>>(s, dt, slot);
+}
+
 // The tuning rule's path (a.path) wins; by default M <= 4 takes the CUDA-core
 // kernel, M <= 128 the weight-streaming kernel, larger M the CTA-pair kernel
-// (the one-CTA kernel if a cluster launch is refused).
+// (operand-swapped for M <= 128; the one-CTA kernel if a cluster launch is
+// refused).
 int launch_tc_bf16(const GemmArgs& a) {
     int path = a.path;
     if (path == PATH_AUTO)
@@ -162,8 +189,9 @@ int launch_tc_bf16(const GemmArgs& a) {
     if (path == PATH_CUDA_CORE) return launch_gemv_bf16(a);
     if (path == PATH_SMALL_M) return launch_skinny_bf16(a);
     if (path == PATH_CTA_PAIR) {
-        const int r = a.stages == 4 ? run_pair<Cfg2BF16s4>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 54)
-                                    : run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
+        const int r = a.M <= kSkinnyMaxM ? run_pair_swapped<1, OutT::BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0, 64)
+                    : a.stages == 4      ? run_pair<Cfg2BF16s4>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 54)
+                                         : run_pair<Cfg2BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3);
         if (r != kUnsupported) return r;
     }
     return run<CfgBF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 0);
@@ -175,8 +203,9 @@ int launch_tc_f16(const GemmArgs& a) {
     if (path == PATH_CUDA_CORE) return launch_gemv_f16(a);
     if (path == PATH_SMALL_M) return launch_skinny_f16(a);
     if (path == PATH_CTA_PAIR) {
-        const int r = a.stages == 4 ? run_pair<Cfg2F16s4>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 55)
-                                    : run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
+        const int r = a.M <= kSkinnyMaxM ? run_pair_swapped<0, OutT::F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 0, 66)
+                    : a.stages == 4      ? run_pair<Cfg2F16s4>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 55)
+                                         : run_pair<Cfg2F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4);
         if (r != kUnsupported) return r;
     }
     return run<CfgF16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1);
@@ -184,13 +213,17 @@ int launch_tc_f16(const GemmArgs& a) {
 // 16-bit GEMM with optionally transposed operands.  Only B transposed (the
 // backward product dA = dC . B^T) follows the plain call's path choice: with
 // M <= 128 and the small-M or CUDA-core path it runs the weight-streaming
-// kernel on K-major weight tiles (there is no transposed CUDA-core kernel).
-// Every other transposed call runs the CTA-pair kernel (no one-CTA variant:
-// a refused cluster launch reports kUnsupported).
+// kernel on K-major weight tiles (there is no transposed CUDA-core kernel),
+// with another path the operand-swapped CTA-pair kernel.  Every other
+// transposed call runs the CTA-pair kernel (no one-CTA variant: a refused
+// cluster launch reports kUnsupported).
 int launch_tc_trans(const GemmArgs& a, int bf16, int trans_a, int trans_b) {
     if (!trans_a && !trans_b) return bf16 ? launch_tc_bf16(a) : launch_tc_f16(a);
     if (!trans_a && a.M <= kSkinnyMaxM && a.path != PATH_CTA_PAIR && a.path != PATH_ONE_CTA)
         return launch_skinny_trans_b(a, bf16);
+    if (!trans_a && a.M <= kSkinnyMaxM)
+        return bf16 ? run_pair_swapped<1, OutT::BF16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, 64)
+                    : run_pair_swapped<0, OutT::F16>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 1, 66);
     const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (bf16) {
         if (trans_a && trans_b) return run_pair<Cfg2T11<1, OutT::BF16>>(a, dt, 11);

@@ -27,6 +27,12 @@
 // possible orders give the same bits).  A half is the last item of its pair,
 // so its operand ring is idle by then: the partial goes out and comes in
 // through the ring by 128 KB bulk copies.
+// Operand-swapped mode (TOUT, 128-column pair tiles) for M <= 128: the
+// caller passes B^T as A and A^T as B, so the kernel computes C^T with the
+// weight columns as its 256-row side and the M activation rows as its
+// 128-column side.  Each CTA then stages 128 weight columns and 64 of the
+// activation rows, where the plain form has one CTA of the pair staging all
+// M rows of A and its partner none; the epilogue writes the tile transposed.
 // Loads are plain tiled TMA copies: each CTA reads only its own tiles into
 // its own shared memory.  Every wait is bounded; the CTAs meet on a cluster
 // barrier after set-up and before freeing TMEM.
@@ -39,7 +45,10 @@ namespace tg {
 // M-major (64-row boxes along M) and the MMA reads A MN-major.  B_MN_ = 0: B
 // is stored transposed (N x K row-major) and is read K-major.  The default
 // (0, 1) is the row-major A (M x K) and B (K x N) of the plain GEMM.
-template <int FMT_, OutT OUT_, int STAGES_, int A_MN_ = 0, int B_MN_ = 1>
+// BN_: columns of a pair tile (256, or 128: each CTA stages 64 B columns).
+// TOUT_ = 1: the kernel computes the transpose D = C^T of the output (the
+// caller swaps the operands) and writes it transposed into C.
+template <int FMT_, OutT OUT_, int STAGES_, int A_MN_ = 0, int B_MN_ = 1, int BN_ = 256, int TOUT_ = 0>
 struct Tc2Cfg {
     static constexpr int FMT = FMT_;
     static constexpr OutT OUT = OUT_;
@@ -48,8 +57,10 @@ struct Tc2Cfg {
     static constexpr int OUT_BYTES = 2;
     static constexpr int BM = 128;                      // rows per CTA
     static constexpr int PM = 256;                      // rows per pair tile
-    static constexpr int BN = 256;                      // columns per pair tile
-    static constexpr int HN = 128;                      // B columns staged per CTA
+    static constexpr int TOUT = TOUT_;
+    static constexpr int BN = BN_;                      // columns per pair tile
+    static constexpr int HN = BN_ / 2;                  // B columns staged per CTA
+    static_assert(BN_ == 256 || BN_ == 128, "pair tile width");
     static constexpr int BK = 64;
     static constexpr int MMA_K = 16;
     static constexpr int STAGES = STAGES_;
@@ -58,6 +69,7 @@ struct Tc2Cfg {
     static constexpr int B_CHUNK = BK * 128;            // 8 KB: 64 columns x 64 rows
     static constexpr int B_STAGE = (HN / 64) * B_CHUNK; // 16 KB
     static constexpr int STG_BUF = 32 * 128;
+    static_assert(STG_BUF == 64 * 64, "a staging buffer holds 32 x 128 bytes or, transposed, 64 x 64");
     static constexpr int EPI_WARPS = 4;
     static constexpr int TMEM_COLS = 2 * BN;            // 512: double-buffered accumulator
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
@@ -67,6 +79,66 @@ struct Tc2Cfg {
     static_assert(STAGES * (A_STAGE + B_STAGE) >= PART_BYTES, "the ring holds a partial");
     static constexpr int SMEM_BYTES = SMEM_DATA + 256 + 1024;
 };
+
+// Epilogue of an operand-swapped tile: the accumulator holds D = C^T (a
+// TMEM lane is a column n of C, a TMEM column a row m of C; p.M and p.N are
+// the kernel's dimensions, N and M of C).  For each 64 rows m, lane n stores
+// its 64 values down column n of a [64 m][32 n] staging tile, so each row of
+// the tile is one contiguous 64-byte run, and one TMA store writes the tile
+// into C at (column n0, row m0): the copy engine drops the rows past M and
+// the columns past N, the latter in whole 16-byte units, so a column tail
+// that is not a whole number of them is written with plain stores instead.
+// The staging buffer is the 4 KB of the plain epilogue.
+template <OutT OUT, int BN, int NBUF>
+__device__ __forceinline__ void epilogue_tile_t(const CUtensorMap* tmC, const TcParams& p,
+                                                uint32_t tmem_tile, int q, int lane,
+                                                int n0, int m_base, uint8_t* stg0,
+                                                uint32_t& nstore) {
+    static_assert(OUT != OutT::F32, "16-bit output");
+    constexpr int STG_BUF = 64 * 64;
+    if (n0 >= p.M) return;                                 // warp-uniform
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+        const int m0 = m_base + 64 * c;
+        if (m0 >= p.N) break;
+        const uint32_t taddr = tmem_tile + (static_cast<uint32_t>(q * 32) << 16) + 64 * c;
+        uint32_t v[64];
+        tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        auto out16 = [&](int j) -> uint16_t {
+            float x = __uint_as_float(v[j]);
+            if (p.relu) x = fmaxf(x, 0.f);
+            if constexpr (OUT == OutT::BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+            else return __half_as_ushort(__float2half_rn(x));
+        };
+        const int ncols = p.M - n0;                        // columns of C left from n0
+        if (ncols < 32 && (ncols * 2) % 16 != 0) {
+            // lane n writes its column; per row the lanes' stores are contiguous
+            if (lane < ncols) {
+                uint16_t* dst = static_cast<uint16_t*>(p.C) + static_cast<long long>(m0) * p.ldc + n0 + lane;
+                const int rows = p.N - m0;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < rows) dst[static_cast<long long>(j) * p.ldc] = out16(j);
+            }
+            continue;
+        }
+        uint8_t* stg = stg0 + (nstore % NBUF) * STG_BUF;
+        if (lane == 0) bulk_wait_read<NBUF - 1>();         // this buffer's last store has read it
+        __syncwarp();
+        uint16_t* col = reinterpret_cast<uint16_t*>(stg) + lane;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) col[32 * j] = out16(j);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmC, stg, n0, m0);
+            bulk_commit();
+        }
+        ++nstore;
+    }
+}
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
@@ -151,7 +223,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 // feed output rows / columns that are never stored
                 // 64-wide chunks (A rows or B columns) that start inside the matrix
                 const int a_live = m0 >= p.M ? 0 : (m0 + 64 < p.M ? 2 : 1);
-                const int b_live = n0 >= p.N ? 0 : (n0 + 64 < p.N ? 2 : 1);
+                const int b_live = n0 >= p.N ? 0 : (Cfg::HN > 64 && n0 + 64 < p.N ? 2 : 1);
                 const uint32_t a_bytes = Cfg::A_MN ? a_live * Cfg::A_CHUNK : (a_live ? Cfg::A_STAGE : 0);
                 const uint32_t b_bytes = Cfg::B_MN ? b_live * Cfg::B_CHUNK : (b_live ? Cfg::B_STAGE : 0);
                 const uint32_t bytes = a_bytes + b_bytes;
@@ -362,9 +434,14 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     }
                 }
             }
-            if (store_tile)
-                epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
-                                                           row0, tn * Cfg::BN, stg0, nstore);
+            if (store_tile) {
+                if constexpr (Cfg::TOUT)
+                    epilogue_tile_t<Cfg::OUT, Cfg::BN, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
+                                                          row0, tn * Cfg::BN, stg0, nstore);
+                else
+                    epilogue_tile<Cfg::OUT, Cfg::BN, false, 2>(&tmC, p, tmem_base + acc * Cfg::BN, q, lane,
+                                                               row0, tn * Cfg::BN, stg0, nstore);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));

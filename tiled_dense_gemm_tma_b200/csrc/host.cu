@@ -45,7 +45,8 @@ std::mutex g_map_mu;
 std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
 constexpr size_t kMaxCachedMaps = 4096;
 
-std::atomic<unsigned long long> g_attr_done[kMaxDevices];
+std::atomic<unsigned long long> g_attr_done[kMaxDevices][kMaxSlots / 64];
+std::atomic<const void*> g_attr_func[kMaxDevices][kMaxSlots];   // the kernel that owns each slot
 
 }  // namespace
 
@@ -147,17 +148,25 @@ cudaError_t set_smem_attr(const void* func, int bytes, int slot) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices || slot < 0 || slot >= 64) return cudaErrorInvalidValue;
-    const unsigned long long bit = 1ull << slot;
-    if (g_attr_done[dev].load(std::memory_order_acquire) & bit) return cudaSuccess;
+    if (dev < 0 || dev >= kMaxDevices || slot < 0 || slot >= kMaxSlots) return cudaErrorInvalidValue;
+    std::atomic<unsigned long long>& done = g_attr_done[dev][slot / 64];
+    const unsigned long long bit = 1ull << (slot % 64);
+    // a slot already set for another kernel is a collision between two
+    // kernels' slot numbers: refuse rather than launch without the attribute
+    if (done.load(std::memory_order_acquire) & bit)
+        return g_attr_func[dev][slot].load(std::memory_order_relaxed) == func ? cudaSuccess
+                                                                             : cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) g_attr_done[dev].fetch_or(bit, std::memory_order_acq_rel);
+    if (e == cudaSuccess) {
+        g_attr_func[dev][slot].store(func, std::memory_order_relaxed);
+        done.fetch_or(bit, std::memory_order_acq_rel);
+    }
     return e;
 }
 
 namespace {
 // -1: not asked yet; indexed [device][slot][log2 S - 1]
-std::atomic<int> g_max_clusters[kMaxDevices][64][3];
+std::atomic<int> g_max_clusters[kMaxDevices][kMaxSlots][3];
 std::once_flag g_max_clusters_once;
 }  // namespace
 
@@ -169,7 +178,7 @@ int max_active_clusters(const void* func, int slot, int S, int threads, int smem
     });
     int dev = 0;
     const int si = S == 2 ? 0 : S == 4 ? 1 : S == 8 ? 2 : -1;
-    if (si < 0 || slot < 0 || slot >= 64 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
+    if (si < 0 || slot < 0 || slot >= kMaxSlots || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
         dev >= kMaxDevices)
         return 0;
     std::atomic<int>& cached = g_max_clusters[dev][slot][si];

@@ -48,8 +48,8 @@ bool pair_kernels_disabled();
 int* device_status_ptr();
 
 // Allow `func` to use `bytes` of dynamic shared memory (once per device).
-// `slot` (0..63) names the kernel in a per-device bitmask of done calls;
-// each kernel instantiation needs its own:
+// `slot` (0..kMaxSlots-1) names the kernel in a per-device bitmask of done
+// calls; each kernel instantiation needs its own:
 //    0-4   gemm_tc.cu        one-CTA bf16/f16/tf32, CTA-pair bf16/f16
 //   54-55  gemm_tc.cu        CTA-pair bf16/f16 with a 4-slot ring (tuning table)
 //    5, 11-15 gemm_tc.cu     CTA-pair with transposed operands
@@ -57,8 +57,11 @@ int* device_status_ptr();
 //    6, 7  gemm_w4a16.cu, gemm_w4a16_pair.cu (FP4 weights)
 //   16-27  gemm_skinny.cu    28-35  gemm_skinny.cu (weights stored transposed)
 //   36-39  gemm_skinny.cu (FP4 weights)
-//   40-48  gemv.cu           50-53  gemm_skinny_static.cu
+//   40-48  gemv.cu           58-60  gemv.cu (FP4 weights)
+//   50-53  gemm_skinny_static.cu
 //   56-57  gemm_sp24.cu (one CTA)   61-62  gemm_sp24.cu (CTA pairs)
+//   64-67  gemm_tc.cu        CTA-pair bf16/f16 with the operands swapped (M <= 128)
+constexpr int kMaxSlots = 128;
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 
 // Clusters of S CTAs (threads and dynamic shared memory bytes each) of the
