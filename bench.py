@@ -546,7 +546,9 @@ SWEEP_CLASSES = [
     ("w4a16", 5, 128, 4096, INF, ["w4a16_gemm_m16"], _SMALL),
     ("w4a16", 129, INF, 1, INF, ["w4a16_gemm_m4096"],
      [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
-    ("wfp4", 1, 128, 4096, INF, ["wfp4_gemm_m1", "wfp4_gemm_m16"], _SMALL),
+    ("wfp4", 1, 4, 4096, INF, ["wfp4_gemm_m1"],
+     [{"path": "cuda_core", "ctas": c} for c in (136, 128, 120, 96)] + [{"path": "small_m"}]),
+    ("wfp4", 5, 128, 4096, INF, ["wfp4_gemm_m16"], _SMALL),
     ("wfp4", 129, INF, 1, INF, ["wfp4_gemm_m4096"],
      [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
     ("f32_ffma", 1, 1024, 1, 1024, ["f32_ffma_gemm_1024"], [{"splits": k} for k in (1, 3, 4)]),

@@ -7,9 +7,8 @@
 namespace tg {
 
 constexpr TuneRule kBuiltinRules[] = {
-    {0, 3, 65, 128, 4096, 0x7fffffffffffffffll, 0, 0, 0, 0},   // bf16 M 65..128: path=cta_pair (0.879 of the default)
-    {2, 1, 1, 4, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 1..4: path=cuda_core, ctas=128 (0.938 of the default)
-    {2, 2, 5, 128, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 5..128: path=small_m, ctas=128 (0.978 of the default)
+    {0, 3, 65, 128, 4096, 0x7fffffffffffffffll, 0, 0, 0, 0},   // bf16 M 65..128: path=cta_pair (0.779 of the default)
+    {2, 2, 5, 128, 4096, 0x7fffffffffffffffll, 128, 0, 0, 0},   // w4a16 M 5..128: path=small_m, ctas=128 (0.967 of the default)
     {-1, 0, 0, 0, 0, 0, 0, 0, 0, 0},   // end: matches nothing
 };
 
