@@ -298,7 +298,9 @@ enum {
     TG_PATH_AUTO = 0,       /* the default choice by M */
     TG_PATH_CUDA_CORE = 1,  /* CUDA-core kernel: M <= 4 only; not for fp32 */
     TG_PATH_SMALL_M = 2,    /* weight-streaming tensor-core kernel: M <= 128 only */
-    TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit and 4-bit ops) */
+    TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit and 4-bit ops;
+                               16-bit calls with M <= 128 run it with the operands
+                               swapped, C^T = B^T A^T, and C written transposed) */
     TG_PATH_ONE_CTA = 4     /* persistent one-CTA tensor-core kernel (not fp32 FFMA) */
 };
 typedef struct {
@@ -311,7 +313,7 @@ typedef struct {
                                capped at the device's SMs; 0 = all */
     int32_t group_m;        /* raster band height in (pair) tiles, 1..256; 0 = default */
     int32_t splits;         /* TG_OP_F32_FFMA only: k ranges per output tile, 1..8 */
-    int32_t stages;         /* 16-bit CTA-pair kernel only: ring depth, 4 or 6 */
+    int32_t stages;         /* 16-bit CTA-pair kernel with M > 128 only: ring depth, 4 or 6 */
 } tg_tune_rule;
 
 /* Replace the run-time rules with `count` rules (at most 64; 0 clears them).
