@@ -63,7 +63,8 @@ CHILD = textwrap.dedent("""
         elif fam.startswith("w4a16") or fam.startswith("skinny_w4a16") or fam.startswith("gemv_w4a16"):
             M, N, K = {"w4a16_pair": (512, 1024, 1024), "w4a16_large": (512, 1024, 1024),
                        "skinny_w4a16": (16, 2048, 4096), "gemv_w4a16": (2, 2048, 8192),
-                       "gemv_w4a16_cluster": (1, 8192, 8192)}[fam]
+                       "gemv_w4a16_cluster": (1, 8192, 8192),
+                       "skinny_w4a16_cluster": (16, 8192, 4096)}[fam]
             A, Bq, S, _ = synth.w4a16(M, N, K, seed=4)
             dA, dB, dS = to_dev(A, "f16"), to_dev(Bq, "u8"), to_dev(S, "f16")
             ref = oracle.gemm_w4a16(A, Bq, S, N=N)
@@ -109,10 +110,11 @@ CHILD = textwrap.dedent("""
     print("RESULT", st, st2, st3, x, round(dt, 3))
 """) % (ROOT, os.path.join(ROOT, "tests"))
 
-# gemv_*_cluster: shapes whose CUDA-core split runs inside clusters (the
-# owners' byte-counting barriers and the closing cluster barrier abort too)
+# *_cluster: shapes whose split-K runs inside clusters (the owners'
+# byte-counting barriers and the closing cluster barrier abort too)
 FAMILIES = ["tc2_bf16", "tf32", "skinny_bf16", "skinny_bf16_tb", "gemv_bf16", "ffma",
-            "ffma_splitk", "w4a16_pair", "skinny_w4a16", "gemv_w4a16", "gemv_w4a16_cluster",
+            "ffma_splitk", "w4a16_pair", "skinny_w4a16", "skinny_w4a16_cluster", "gemv_w4a16",
+            "gemv_w4a16_cluster",
             "wfp4_pair", "skinny_wfp4", "gemv_wfp4", "gemv_wfp4_cluster", "sp24_pair", "tc_bf16",
             "w4a16_large", "wfp4_large", "sp24_one"]
 # run with the CTA-pair kernels off

@@ -23,8 +23,8 @@
 //   group's last segment (counted with an atomic ticket) sums the partials
 //   in segment order -- deterministic -- applies ReLU, rounds and writes C,
 //   and resets the ticket for the next call.
-// * Split-K inside clusters (16-bit weights, where T groups times a split S
-//   in {8, 4, 2, 1} fill at least three quarters of the SMs): group t goes to
+// * Split-K inside clusters (where T groups times a split S in {8, 4, 2, 1}
+//   fill at least three quarters of the SMs): group t goes to
 //   the S CTAs of cluster t, each taking a contiguous part of its k-units.
 //   When its accumulator is final a CTA's ring is idle; the ranks exchange
 //   "ring free" signals, store their partials of each rank's GN/S columns
@@ -674,12 +674,13 @@ skinny_kernel(const __grid_constant__ CUtensorMap tmW,
 // Host side, shared by the regular and the static entry points.  The
 // cluster split of cl_split for T column groups of KB k-units, lowered until
 // the device holds all T clusters of that size at once; 0 selects stream-K.
-// 4-bit weights always take stream-K: their pace is set per SM (expanding
-// the packed weights), so they need every SM, which the split into T*S CTAs
-// seldom gives.  `slot` is the kernel's attribute slot (set_smem_attr done).
+// 4-bit weights too: their pace is set per SM (expanding the packed
+// weights), so the split's T*S CTAs leave SMs idle, but the cluster
+// reduction costs less than stream-K's tail through global memory.  `slot`
+// is the kernel's attribute slot (set_smem_attr done).
 template <class Cfg>
 inline int skinny_cluster_split(long long T, long long KB, long long cap, int num_sms, int slot) {
-    if constexpr (!Cfg::CL_OK || Cfg::Q4) {
+    if constexpr (!Cfg::CL_OK) {
         return 0;
     } else {
         const void* k = reinterpret_cast<const void*>(skinny_kernel<Cfg>);
