@@ -56,7 +56,7 @@ int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, 
     const long long ntn = (a.N + Cfg::BN - 1) / Cfg::BN;
     const long long tiles = ntm * ntn;
     const int grid = static_cast<int>(persistent_grid(tiles, di->num_sms, a.ctas));
-    TcParams p;
+    TcParams p = {};
     p.M = static_cast<int>(a.M);
     p.N = static_cast<int>(a.N);
     p.K = static_cast<int>(a.K);
