@@ -40,18 +40,17 @@
  *   split-K workspace per (device, stream): fp32 partials and tile tickets
  *   of the kernels that split K across CTAs through global memory (small M
  *   where the split does not run inside thread-block clusters, fp32 shapes
- *   with fewer 128 x 128 tiles than SMs, and 16-bit GEMMs with M > 128 whose
- *   last wave of 256 x 256 tiles is split along K).  It is allocated on the
- *   first such call on a stream (at least 8 MiB), grown when a larger call
- *   needs it (the
- *   regrow frees the old one, which synchronises the device), and reused.
- *   Calls on one stream share it; calls on different streams get their own
- *   (cudaStreamPerThread counts as one stream per host thread).  A stream
- *   under CUDA graph capture never allocates it: there the 16-bit GEMM with
- *   M > 128 runs its last wave of tiles whole, and the other users of the
- *   workspace return TG_ERR_CUDA unless one uncaptured call of the largest
- *   shape on that stream came first.  tg_gemm_bf16_small_m_static avoids
- *   it.
+ *   with fewer 128 x 128 tiles than SMs, and 16-bit GEMMs on the CTA-pair
+ *   kernel whose last wave of tiles is split along K).  It is allocated on
+ *   the first such call on a stream (at least 8 MiB), grown when a larger
+ *   call needs it (the regrow frees the old one, which synchronises the
+ *   device), and reused.  Calls on one stream share it; calls on different
+ *   streams get their own (cudaStreamPerThread counts as one stream per
+ *   host thread).  A stream under CUDA graph capture never allocates it:
+ *   there the 16-bit GEMM on the CTA-pair kernel runs its last wave of
+ *   tiles whole, and the other users of the workspace return TG_ERR_CUDA
+ *   unless one uncaptured call of the largest shape on that stream came
+ *   first.  tg_gemm_bf16_small_m_static avoids it.
  * - Thread safety: calls from several host threads are allowed.  A thread
  *   needs no earlier CUDA call: on its first call the library makes the
  *   current device's primary context current on that thread.
