@@ -552,7 +552,8 @@ SWEEP_CLASSES = [
     ("wfp4", 129, INF, 1, INF, ["wfp4_gemm_m4096"],
      [{"path": "cta_pair", "group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
     ("f32_ffma", 1, 1024, 1, 1024, ["f32_ffma_gemm_1024"], [{"splits": k} for k in (1, 3, 4)]),
-    ("f32_tf32", 129, INF, 1, INF, ["f32_tf32_gemm_4096"], [{"group_m": g} for g in (8, 32)]),
+    ("f32_tf32", 129, INF, 1, INF, ["f32_tf32_gemm_4096"],
+     [{"group_m": g} for g in (4, 16)] + [{"path": "one_cta"}]),
 ]
 SWEEP_MARGIN = 0.02
 TUNE_TABLE = os.path.join(ROOT, "tiled_dense_gemm_tma_b200", "csrc", "tune_table.h")

@@ -88,7 +88,9 @@ enum { TG_EPI_NONE = 0, TG_EPI_RELU = 1 };
 enum {
     TG_F32_FFMA = 0,  /* exact fp32 products, fp32 FMA accumulation on CUDA cores */
     TG_F32_TF32 = 1   /* operands rounded to TF32 (10-bit mantissa) by the tensor
-                         cores, fp32 accumulation in tensor memory */
+                         cores, fp32 accumulation in tensor memory; M > 128 on
+                         CTA pairs (256 x 256 tiles), M <= 128 (or a refused
+                         cluster launch) on one CTA per SM (128 x 256 tiles) */
 };
 
 /*
@@ -297,9 +299,10 @@ enum {
     TG_PATH_AUTO = 0,       /* the default choice by M */
     TG_PATH_CUDA_CORE = 1,  /* CUDA-core kernel: M <= 4 only; not for fp32 */
     TG_PATH_SMALL_M = 2,    /* weight-streaming tensor-core kernel: M <= 128 only */
-    TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit and 4-bit ops;
-                               16-bit calls with M <= 128 run it with the operands
-                               swapped, C^T = B^T A^T, and C written transposed) */
+    TG_PATH_CTA_PAIR = 3,   /* persistent CTA-pair tensor-core kernel (16-bit, 4-bit and
+                               TF32 ops; 16-bit calls with M <= 128 run it with the
+                               operands swapped, C^T = B^T A^T, and C written
+                               transposed) */
     TG_PATH_ONE_CTA = 4     /* persistent one-CTA tensor-core kernel (not fp32 FFMA) */
 };
 typedef struct {

@@ -214,6 +214,36 @@ def test_tf32_integer_bit_exact(tg):
     assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(A, B, relu=True)))
 
 
+@pytest.mark.parametrize("shape", [(512, 768, 384), (129, 127, 1000), (2048, 7400, 100)])
+def test_tf32_one_cta_forced(tg, shape):
+    # TF32 with M > 128 runs on CTA pairs; the one-CTA kernel (M <= 128, and
+    # the path when a cluster launch is refused) forced by a tuning rule,
+    # including more tiles than CTAs (2048 x 7400: 464 tiles of 128 x 256)
+    M, N, K = shape
+    A, B = synth.normal(M, N, K, seed=1)
+    tg.tune_set([{"op": "f32_tf32", "path": "one_cta"}])
+    try:
+        for relu in (False, True):
+            got = _run_f32(tg, A, B, tg.F32_TF32, relu=relu)
+            assert rel_frob(got, oracle.gemm_f32(A, B, relu)) <= 5e-3
+        Ai, Bi = synth.integers(M, N, K, seed=1)
+        got = _run_f32(tg, Ai, Bi, tg.F32_TF32)
+        assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(Ai, Bi)))
+    finally:
+        tg.tune_set([])
+
+
+def test_tf32_pair_forced_small_m(tg):
+    # a CTA-pair rule for M <= 128: the partner CTA of every pair has no rows
+    A, B = synth.integers(100, 1000, 520, seed=2)
+    tg.tune_set([{"op": "f32_tf32", "path": "cta_pair"}])
+    try:
+        got = _run_f32(tg, A, B, tg.F32_TF32)
+        assert np.array_equal(got, oracle.round_f32(oracle.gemm_f32(A, B)))
+    finally:
+        tg.tune_set([])
+
+
 # ------------------------------------------- small M: weight-streaming kernel
 
 SKINNY = [(1, 1000, 640), (2, 384, 4096), (16, 2048, 1000), (17, 520, 333), (33, 1024, 2048),

@@ -30,6 +30,8 @@ template <int FMT, OutT OUT>
 using Cfg2S = Tc2Cfg<FMT, OUT, 6, 1, 0, 128, 1>;
 template <int FMT, OutT OUT>
 using Cfg2ST = Tc2Cfg<FMT, OUT, 6, 0, 0, 128, 1>;
+// TF32 mode on CTA pairs (M > 128)
+using Cfg2TF32 = Tc2Cfg<2, OutT::F32, 6>;
 
 template <class Cfg>
 int run(const GemmArgs& a, CUtensorMapDataType in_t, CUtensorMapDataType out_t, int slot) {
@@ -85,21 +87,25 @@ int run_pair(const GemmArgs& a, CUtensorMapDataType dt, int slot) {
     const DeviceInfo* di = current_device(&dev);
     if (!di) return kNoDevice;
     CUtensorMap tA, tB, tC;
-    // A: row-major M x K -> K-major boxes of BK x BM rows; stored transposed
-    // (K x M) -> M-major boxes of 64 rows of A x BK.
-    if (Cfg::A_MN ? !tensor_map_2d(&tA, a.A, dt, 2, a.M, a.K, a.lda * 2, 64, Cfg::BK, SWZ_128)
-                  : !tensor_map_2d(&tA, a.A, dt, 2, a.K, a.M, a.lda * 2, Cfg::BK, Cfg::BM, SWZ_128))
+    constexpr int eb = Cfg::IN_BYTES, ob = Cfg::OUT_BYTES;
+    const CUtensorMapDataType ot = Cfg::OUT == OutT::F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : dt;
+    // A: row-major M x K -> K-major boxes of BK (128 B) x BM rows; stored
+    // transposed (K x M) -> M-major boxes of 64 rows of A x BK.
+    if (Cfg::A_MN ? !tensor_map_2d(&tA, a.A, dt, eb, a.M, a.K, a.lda * eb, 64, Cfg::BK, SWZ_128)
+                  : !tensor_map_2d(&tA, a.A, dt, eb, a.K, a.M, a.lda * eb, Cfg::BK, Cfg::BM, SWZ_128))
         return kCudaError;
-    // B: row-major K x N -> N-major boxes of 64 columns x BK; stored
-    // transposed (N x K) -> K-major boxes of BK x HN columns.
-    if (Cfg::B_MN ? !tensor_map_2d(&tB, a.B, dt, 2, a.N, a.K, a.ldb * 2, 64, Cfg::BK, SWZ_128)
-                  : !tensor_map_2d(&tB, a.B, dt, 2, a.K, a.N, a.ldb * 2, Cfg::BK, Cfg::HN, SWZ_128))
+    // B: row-major K x N -> N-major boxes of CHUNK_N (128 B) columns x BK
+    // (32-bit data with the 32-byte-unit swizzle); stored transposed (N x K)
+    // -> K-major boxes of BK x HN columns.
+    if (Cfg::B_MN ? !tensor_map_2d(&tB, a.B, dt, eb, a.N, a.K, a.ldb * eb, Cfg::CHUNK_N, Cfg::BK,
+                                   eb == 4 ? SWZ_128_32B : SWZ_128)
+                  : !tensor_map_2d(&tB, a.B, dt, eb, a.K, a.N, a.ldb * eb, Cfg::BK, Cfg::HN, SWZ_128))
         return kCudaError;
-    // C: 64-column x 32-row boxes of the tile; in the operand-swapped mode the
+    // C: 128-byte x 32-row boxes of the tile; in the operand-swapped mode the
     // kernel's M x N is C^T, and C (a.N rows x a.M columns) takes unswizzled
     // boxes of 32 columns x 64 rows
-    if (Cfg::TOUT ? !tensor_map_2d(&tC, a.C, dt, 2, a.M, a.N, a.ldc * 2, 32, 64, SWZ_NONE)
-                  : !tensor_map_2d(&tC, a.C, dt, 2, a.N, a.M, a.ldc * 2, 64, 32, SWZ_128))
+    if (Cfg::TOUT ? !tensor_map_2d(&tC, a.C, ot, ob, a.M, a.N, a.ldc * ob, 32, 64, SWZ_NONE)
+                  : !tensor_map_2d(&tC, a.C, ot, ob, a.N, a.M, a.ldc * ob, 128 / ob, 32, SWZ_128))
         return kCudaError;
     auto kern = tc2_gemm_kernel<Cfg>;
     if (set_smem_attr(reinterpret_cast<const void*>(kern), Cfg::SMEM_BYTES, slot) != cudaSuccess)
@@ -233,7 +239,16 @@ int launch_tc_trans(const GemmArgs& a, int bf16, int trans_a, int trans_b) {
     return trans_a ? run_pair<Cfg2T10<0, OutT::F16>>(a, dt, 15) : run_pair<Cfg2T01<0, OutT::F16>>(a, dt, 5);
 }
 
+// TF32 mode: M > 128 on CTA pairs by default (the one-CTA kernel if a
+// cluster launch is refused); M <= 128, or a one-CTA tuning rule, on the
+// one-CTA kernel.
 int launch_tc_tf32(const GemmArgs& a) {
+    int path = a.path;
+    if (path == PATH_AUTO) path = a.M <= kSkinnyMaxM ? PATH_ONE_CTA : PATH_CTA_PAIR;
+    if (path == PATH_CTA_PAIR) {
+        const int r = run_pair<Cfg2TF32>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 68);
+        if (r != kUnsupported) return r;
+    }
     return run<CfgTF32>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2);
 }
 

@@ -1,4 +1,5 @@
-// gemm_tc2.cuh -- the fp16 / bf16 GEMM on CTA pairs (tcgen05 cta_group::2).
+// gemm_tc2.cuh -- the fp16 / bf16 GEMM and the TF32 mode of the fp32 GEMM
+// on CTA pairs (tcgen05 cta_group::2).
 //
 // Same warp roles as gemm_tc.cuh, but two CTAs on neighbouring SMs (a
 // cluster of 2) share one 256 x 256 output tile: CTA rank r owns rows
@@ -8,7 +9,10 @@
 // SMs read A from their own CTA and B from both, and each CTA's TMEM receives
 // its 128 rows x 256 columns.  Per MMA each SM reads 4 KB of A and 4 KB of B
 // from its shared memory instead of 4 KB + 8 KB in the single-CTA kernel,
-// which relieves the shared-memory -> tensor-core path.
+// which relieves the shared-memory -> tensor-core path.  TF32 (fp32
+// operands, kind::tf32, fp32 output): the same 128-byte rows hold 32 k, B
+// arrives in 32-column boxes with the 32-byte-unit swizzle the tensor core
+// requires for MN-major 32-bit data, and each MMA covers 8 k.
 //
 // Synchronisation across the pair:
 //   full[s]   leader only; both producers arm it (count 2) with their own byte
@@ -50,24 +54,32 @@ namespace tg {
 // caller swaps the operands) and writes it transposed into C.
 template <int FMT_, OutT OUT_, int STAGES_, int A_MN_ = 0, int B_MN_ = 1, int BN_ = 256, int TOUT_ = 0>
 struct Tc2Cfg {
-    static constexpr int FMT = FMT_;
+    static constexpr int FMT = FMT_;                    // idesc format: 0 f16, 1 bf16, 2 tf32
     static constexpr OutT OUT = OUT_;
     static constexpr int A_MN = A_MN_;
     static constexpr int B_MN = B_MN_;
-    static constexpr int OUT_BYTES = 2;
+    static constexpr int IN_BYTES = FMT_ == 2 ? 4 : 2;
+    static constexpr int OUT_BYTES = OUT_ == OutT::F32 ? 4 : 2;
     static constexpr int BM = 128;                      // rows per CTA
     static constexpr int PM = 256;                      // rows per pair tile
     static constexpr int TOUT = TOUT_;
     static constexpr int BN = BN_;                      // columns per pair tile
     static constexpr int HN = BN_ / 2;                  // B columns staged per CTA
     static_assert(BN_ == 256 || BN_ == 128, "pair tile width");
-    static constexpr int BK = 64;
-    static constexpr int MMA_K = 16;
+    // TF32: the plain layout only (A M x K, B K x N, 256-column tiles), fp32 out
+    static_assert(FMT_ != 2 || (A_MN_ == 0 && B_MN_ == 1 && BN_ == 256 && TOUT_ == 0 && OUT_ == OutT::F32),
+                  "TF32 pair configuration");
+    static constexpr int BK = 128 / IN_BYTES;           // k per 128-byte swizzle row: 64 or 32
+    static constexpr int MMA_K = 32 / IN_BYTES;         // k per MMA: 16 or 8
+    static constexpr int CHUNK_N = 128 / IN_BYTES;      // B columns per MN-major box row
     static constexpr int STAGES = STAGES_;
     static constexpr int A_STAGE = BM * 128;            // 16 KB
     static constexpr int A_CHUNK = BK * 128;            // 8 KB: 64 rows of A x 64 k (M-major A)
-    static constexpr int B_CHUNK = BK * 128;            // 8 KB: 64 columns x 64 rows
-    static constexpr int B_STAGE = (HN / 64) * B_CHUNK; // 16 KB
+    static constexpr int B_CHUNK = BK * 128;            // CHUNK_N columns x BK rows: 8 KB / 4 KB
+    static constexpr int B_STAGE = (HN / CHUNK_N) * B_CHUNK;   // 16 KB (K-major B: HN rows x 128 B)
+    // MN-major B: 16-bit data in the 8-row swizzle atom, tf32 in the 4-row one
+    static constexpr uint32_t B_LAYOUT = IN_BYTES == 4 ? 1u : 2u;
+    static constexpr uint32_t B_SBO = IN_BYTES == 4 ? 512u : 1024u;
     static constexpr int STG_BUF = 32 * 128;
     static_assert(STG_BUF == 64 * 64, "a staging buffer holds 32 x 128 bytes or, transposed, 64 x 64");
     static constexpr int EPI_WARPS = 4;
@@ -221,9 +233,11 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 const int n0 = tn * Cfg::BN + rank * Cfg::HN;
                 // boxes entirely past the matrix edge are not loaded: they only
                 // feed output rows / columns that are never stored
-                // 64-wide chunks (A rows or B columns) that start inside the matrix
+                // 64-wide chunks of A rows, CHUNK_N-wide chunks of B columns,
+                // that start inside the matrix
                 const int a_live = m0 >= p.M ? 0 : (m0 + 64 < p.M ? 2 : 1);
-                const int b_live = n0 >= p.N ? 0 : (Cfg::HN > 64 && n0 + 64 < p.N ? 2 : 1);
+                const int b_left = (p.N - n0 + Cfg::CHUNK_N - 1) / Cfg::CHUNK_N;
+                const int b_live = n0 >= p.N ? 0 : (b_left < Cfg::HN / Cfg::CHUNK_N ? b_left : Cfg::HN / Cfg::CHUNK_N);
                 const uint32_t a_bytes = Cfg::A_MN ? a_live * Cfg::A_CHUNK : (a_live ? Cfg::A_STAGE : 0);
                 const uint32_t b_bytes = Cfg::B_MN ? b_live * Cfg::B_CHUNK : (b_live ? Cfg::B_STAGE : 0);
                 const uint32_t bytes = a_bytes + b_bytes;
@@ -246,7 +260,7 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     if constexpr (Cfg::B_MN) {
                         for (int j = 0; j < b_live; ++j)
                             tma_load_2d_pair(smB + s * Cfg::B_STAGE + j * Cfg::B_CHUNK, &tmB, fbar,
-                                             n0 + 64 * j, kb * Cfg::BK);
+                                             n0 + Cfg::CHUNK_N * j, kb * Cfg::BK);
                     } else if (b_live) {                      // stored N x K: one box of 128 columns
                         tma_load_2d_pair(smB + s * Cfg::B_STAGE, &tmB, fbar, kb * Cfg::BK, n0);
                     }
@@ -291,15 +305,18 @@ tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const uint32_t b_addr = smem_u32(smB + s * Cfg::B_STAGE);
 #pragma unroll
                     for (int k = 0; k < Cfg::BK / Cfg::MMA_K; ++k) {
-                        // K-major: 16 k = 32 bytes along a 128-byte row; MN-major: 16 k
-                        // rows of 128 bytes, 64-wide chunks LBO apart
+                        // K-major: MMA_K k = 32 bytes along a 128-byte row; MN-major:
+                        // MMA_K rows of 128 bytes, chunks LBO apart
                         const uint64_t ad = Cfg::A_MN
                             ? sw128_desc(a_addr + k * Cfg::MMA_K * 128, Cfg::A_CHUNK, 1024)
                             : sw128_desc(a_addr + k * 32, 16, 1024);
                         const uint64_t bd = Cfg::B_MN
-                            ? sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, 1024)
+                            ? sw128_desc(b_addr + k * Cfg::MMA_K * 128, Cfg::B_CHUNK, Cfg::B_SBO, Cfg::B_LAYOUT)
                             : sw128_desc(b_addr + k * 32, 16, 1024);
-                        mma_f16_pair(d_tmem, ad, bd, idesc, (kb != kb0) || k != 0);
+                        if constexpr (Cfg::FMT == 2)
+                            mma_tf32_pair(d_tmem, ad, bd, idesc, (kb != kb0) || k != 0);
+                        else
+                            mma_f16_pair(d_tmem, ad, bd, idesc, (kb != kb0) || k != 0);
                     }
                     const uint32_t e_loc = smem_u32(&empty[s]);
                     mma_commit_pair(mapa_shared(e_loc, 0));      // both CTAs' slots

@@ -61,6 +61,7 @@ int* device_status_ptr();
 //   50-53  gemm_skinny_static.cu
 //   56-57  gemm_sp24.cu (one CTA)   61-62  gemm_sp24.cu (CTA pairs)
 //   64-67  gemm_tc.cu        CTA-pair bf16/f16 with the operands swapped (M <= 128)
+//   68     gemm_tc.cu        CTA-pair TF32
 constexpr int kMaxSlots = 128;
 cudaError_t set_smem_attr(const void* func, int bytes, int slot);
 

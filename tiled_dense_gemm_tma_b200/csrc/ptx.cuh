@@ -478,6 +478,17 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
+// The same with kind::tf32 (fp32 operands, tf32 arithmetic; K = 8 per MMA).
+__device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // The sparse form on CTA pairs: A (both CTAs' shared memory, compressed,
 // M split) with each CTA's position codes in its own tensor memory at the
 // same address e_tmem.

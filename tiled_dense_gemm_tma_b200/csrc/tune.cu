@@ -49,7 +49,7 @@ bool tune_rule_valid(const TuneRule& r) {
         case PATH_AUTO: return true;
         case PATH_CUDA_CORE: return !fp32 && r.m_hi <= 4;
         case PATH_SMALL_M: return !fp32 && r.m_hi <= 128;
-        case PATH_CTA_PAIR: return !fp32;
+        case PATH_CTA_PAIR: return r.op != OP_F32_FFMA;
         case PATH_ONE_CTA: return r.op != OP_F32_FFMA;
         default: return false;
     }
