@@ -268,18 +268,26 @@ def test_tuning_table_rules(lib):
         rules = [{"op": "bf16", "path": "small_m", "m_lo": 5, "m_hi": 64, "ctas": 100},
                  {"op": "bf16", "path": "cta_pair", "m_lo": 1, "m_hi": 1 << 40, "stages": 4,
                   "group_m": 4},
-                 {"op": "f32_ffma", "splits": 3}]
+                 {"op": "f32_ffma", "splits": 3},
+                 {"op": "f32_tf32", "path": "one_cta", "m_lo": 129, "m_hi": 4096},
+                 {"op": "f32_tf32", "path": "cta_pair", "m_lo": 1, "m_hi": 128}]
         b.tune_set(rules)
         q = b.tune_query("bf16", 16, 8192)
         assert (q["path"], q["ctas"]) == (b.PATHS["small_m"], 100)        # first match wins
         q = b.tune_query("bf16", 65, 8192)
         assert (q["path"], q["stages"], q["group_m"]) == (b.PATHS["cta_pair"], 4, 4)
         assert b.tune_query("f32_ffma", 1024, 1024)["splits"] == 3
+        # TF32 runs on either tensor-core kernel, by rule
+        assert b.tune_query("f32_tf32", 4096, 4096)["path"] == b.PATHS["one_cta"]
+        assert b.tune_query("f32_tf32", 100, 4096)["path"] == b.PATHS["cta_pair"]
         # malformed rules: nothing changes
         bad = [{"op": "bf16", "path": "cuda_core", "m_hi": 5},       # CUDA-core kernel: M <= 4
                {"op": "wfp4", "path": "cuda_core", "m_hi": 5},        # CUDA-core FP4 kernel: M <= 4
                {"op": "bf16", "path": "small_m", "m_hi": 129},        # small-M kernel: M <= 128
                {"op": "f32_ffma", "path": "one_cta"},                 # fp32 FFMA has one kernel
+               {"op": "f32_ffma", "path": "cta_pair"},
+               {"op": "f32_tf32", "path": "small_m", "m_hi": 128},    # no fp32 small-M kernel
+               {"op": "f32_tf32", "path": "cuda_core", "m_hi": 4},
                {"op": "bf16", "splits": 2},                           # split count: FFMA only
                {"op": "w4a16", "stages": 4},                          # ring depth: 16-bit pair only
                {"op": "bf16", "stages": 5},
