@@ -50,13 +50,13 @@ CHILD = textwrap.dedent("""
             call = lambda: tg.gemm_bf16(dA, dB, trans_b=tb)
             conv = lambda C: decode16(from_dev(C, "bf16"), "bf16")
             tol = (1e-2, 1e-2)
-        elif fam in ("ffma", "ffma_splitk", "tf32"):
+        elif fam in ("ffma", "ffma_splitk", "tf32", "tf32_one"):
             M, N, K = {"ffma": (2048, 1024, 256), "ffma_splitk": (200, 200, 3000),
-                       "tf32": (512, 768, 512)}[fam]
+                       "tf32": (512, 768, 512), "tf32_one": (512, 768, 512)}[fam]
             A, B = synth.normal(M, N, K, seed=1)
             dA, dB = to_dev(A, "f32"), to_dev(B, "f32")
             ref = oracle.gemm_f32(A, B)
-            mode = tg.F32_TF32 if fam == "tf32" else tg.F32_FFMA
+            mode = tg.F32_TF32 if fam.startswith("tf32") else tg.F32_FFMA
             call = lambda: tg.gemm_f32(dA, dB, mode=mode)
             conv = lambda C: from_dev(C, "f32")
             tol = None
@@ -91,7 +91,7 @@ CHILD = textwrap.dedent("""
         def check(C):
             got = conv(C)
             if tol is None:
-                assert rel_frob(got, ref) <= (5e-3 if fam == "tf32" else 1e-5), fam
+                assert rel_frob(got, ref) <= (5e-3 if fam.startswith("tf32") else 1e-5), fam
             else:
                 assert_close(got, ref, tol[0], tol[1], fam)
         return call, check
@@ -116,9 +116,9 @@ FAMILIES = ["tc2_bf16", "tf32", "skinny_bf16", "skinny_bf16_tb", "gemv_bf16", "f
             "ffma_splitk", "w4a16_pair", "skinny_w4a16", "skinny_w4a16_cluster", "gemv_w4a16",
             "gemv_w4a16_cluster",
             "wfp4_pair", "skinny_wfp4", "gemv_wfp4", "gemv_wfp4_cluster", "sp24_pair", "tc_bf16",
-            "w4a16_large", "wfp4_large", "sp24_one"]
+            "w4a16_large", "wfp4_large", "sp24_one", "tf32_one"]
 # run with the CTA-pair kernels off
-ONE_CTA = {"tc_bf16", "w4a16_large", "wfp4_large", "sp24_one"}
+ONE_CTA = {"tc_bf16", "w4a16_large", "wfp4_large", "sp24_one", "tf32_one"}
 
 
 @pytest.mark.parametrize("family", FAMILIES)
