@@ -45,7 +45,7 @@ namespace {
 
 struct W4P {
     static constexpr int BM = 128, PM = 256, BN = 256, HN = 128, BK = 64;
-    static constexpr int STAGES = 6, B_STAGES = 3;
+    static constexpr int STAGES = 6, B_STAGES = 4;
     static constexpr int A_STAGE = BM * BK * 2;          // 16 KB
     static constexpr int Q_BYTES = BK * HN / 2;          // 4 KB packed
     static constexpr int S_BYTES = HN * 2;               // 256 B scales
